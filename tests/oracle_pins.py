@@ -1,0 +1,236 @@
+"""Pins that tie the fp64 oracle to facts other than itself.
+
+Each pin takes a loaded oracle library (the real one, or a deliberately broken
+build made by the mutation test) and raises AssertionError when the oracle
+disagrees with:
+  * brute force over all K^L code combinations (greedy = lexicographic minimiser
+    of (d_0, id_0, d_1, id_1, ...)),
+  * a library nearest-neighbour search (scipy cdist + argmin) when L = 1,
+  * closed forms (K = 1; codebook = the features; planted codewords with a wide
+    margin; integer-valued decode),
+  * invariants (recon + residual == x; residual norms never grow when every level
+    holds a zero codeword; exact ties go to the lowest index),
+  * the hand-worked example in tests/golden/rvq_toy_2d.txt.
+"""
+from __future__ import annotations
+
+import itertools
+import os
+
+import numpy as np
+from scipy.spatial.distance import cdist
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def brute_force_greedy(x, C):
+    """All K^L combinations; returns the lexicographic minimiser of (d_0,id_0,d_1,id_1,...)."""
+    x = np.asarray(x, np.float64)
+    C = np.asarray(C, np.float64)
+    L, K, D = C.shape
+    out = np.empty((x.shape[0], L), np.int32)
+    for n in range(x.shape[0]):
+        best_key = None
+        for combo in itertools.product(range(K), repeat=L):
+            r = x[n].copy()
+            key = []
+            for l, k in enumerate(combo):
+                diff = r - C[l, k]
+                key += [float(np.dot(diff, diff)), k]
+                r = diff
+            key = tuple(key)
+            if best_key is None or key < best_key:
+                best_key, best = key, combo
+        out[n] = best
+    return out
+
+
+def pin_bruteforce(lib):
+    for seed, (N, D, L, K) in enumerate([(24, 3, 2, 5), (16, 8, 3, 4), (32, 2, 2, 8), (8, 5, 3, 7)]):
+        rng = _rng(100 + seed)
+        C = rng.standard_normal((L, K, D)).astype(np.float32)
+        C *= (0.6 ** np.arange(L, dtype=np.float32))[:, None, None]
+        x = rng.standard_normal((N, D)).astype(np.float32)
+        ids, _, _, _ = oracle.encode(x, C, lib=lib)
+        ref = brute_force_greedy(x, C)
+        assert np.array_equal(ids, ref), f"brute force mismatch (case {seed})"
+
+
+def pin_nearest_neighbour_L1(lib):
+    rng = _rng(7)
+    for N, D, K in [(200, 16, 64), (64, 1, 33), (50, 130, 9)]:
+        C = rng.standard_normal((1, K, D)).astype(np.float32)
+        x = rng.standard_normal((N, D)).astype(np.float32)
+        ids, res, rec, dist = oracle.encode(x, C, lib=lib)
+        dm = cdist(x.astype(np.float64), C[0].astype(np.float64), "sqeuclidean")
+        assert np.array_equal(ids[:, 0], np.argmin(dm, axis=1)), "L=1 is not plain nearest neighbour"
+        assert np.allclose(dist[:, 0], dm.min(axis=1), rtol=1e-12, atol=1e-12)
+        assert np.allclose(rec, C[0][ids[:, 0]], rtol=0, atol=0)
+
+
+def pin_single_codeword(lib):
+    rng = _rng(8)
+    C = rng.standard_normal((3, 1, 6)).astype(np.float32)
+    x = rng.standard_normal((10, 6)).astype(np.float32)
+    ids, res, rec, dist = oracle.encode(x, C, lib=lib)
+    assert (ids == 0).all()
+    expect_res = x.astype(np.float64) - C[0, 0] - C[1, 0] - C[2, 0]
+    assert np.allclose(res, expect_res, rtol=1e-15, atol=1e-15)
+    assert np.allclose(rec, C[:, 0].astype(np.float64).sum(0), rtol=1e-15, atol=1e-15)
+
+
+def pin_codebook_equals_features(lib):
+    rng = _rng(9)
+    x = rng.standard_normal((40, 12)).astype(np.float32)
+    perm = rng.permutation(40)
+    C = x[perm][None]                     # codeword perm^-1(n) is row n exactly
+    ids, res, rec, dist = oracle.encode(x, C, lib=lib)
+    inv = np.argsort(perm)
+    assert np.array_equal(ids[:, 0], inv)
+    assert (dist == 0).all() and (res == 0).all()
+
+
+def pin_ties_lowest_index(lib):
+    rng = _rng(10)
+    base = rng.standard_normal((6, 4)).astype(np.float32)
+    C = np.concatenate([base, base, base])[None]        # every codeword appears 3 times
+    C = C[:, rng.permutation(18)]
+    x = rng.standard_normal((30, 4)).astype(np.float32)
+    ids, _, _, _ = oracle.encode(x, C, lib=lib)
+    for n in range(30):
+        same = np.where((C[0] == C[0][ids[n, 0]]).all(axis=1))[0]
+        assert ids[n, 0] == same.min(), "exact tie not broken to the lowest index"
+    # an exact geometric tie: x equidistant from two distinct codewords
+    C2 = np.array([[[3, 0], [-1, 0], [1, 0]]], np.float32)
+    x2 = np.array([[0, 0], [2, 0]], np.float32)            # d=(9,1,1) and (1,9,1)
+    ids2, _, _, _ = oracle.encode(x2, C2, lib=lib)
+    assert ids2[:, 0].tolist() == [1, 0]
+
+
+def pin_invariants(lib):
+    g = workloads.generate("tiny")
+    x, C = g["x"], g["codebooks"]
+    ids, res, rec, dist = oracle.encode(x, C, lib=lib)
+    xd = x.astype(np.float64)
+    err = np.abs(rec + res - xd).max() / np.abs(xd).max()
+    assert err <= 1e-12, f"recon + residual != x ({err})"
+    # every level has a zero codeword, so ||r_{l+1}||^2 = dist[l] <= ||r_l||^2
+    prev = (xd ** 2).sum(1)
+    for l in range(C.shape[0]):
+        assert (dist[:, l] <= prev * (1 + 1e-15)).all(), "residual norm grew"
+        prev = dist[:, l]
+    assert np.allclose(dist[:, -1], (res ** 2).sum(1), rtol=1e-12)
+    # the recon of the chosen ids is the decode of those ids
+    assert np.allclose(oracle.decode(ids, C, lib=lib), rec, rtol=0, atol=1e-12)
+
+
+def pin_planted(lib):
+    # level-0 planted codeword beats any other by ~2*D*1 against noise ~2*sqrt(2*D*sum_rest)
+    g = workloads.generate("image", n_override=48)
+    x, C, planted = g["x"], g["codebooks"], g["planted"]
+    C0 = C[:1]
+    ids, _, _, _ = oracle.encode(x, C0, lib=lib)
+    assert np.array_equal(ids[:, 0], planted[:, 0]), "planted level-0 codeword not recovered"
+    # noiseless round trip (detok recipe, shrunk): decode then re-encode returns the ids
+    rng = _rng(11)
+    L, K, D = 3, 64, 96
+    Cb = workloads.round_bf16(rng.standard_normal((L, K, D)).astype(np.float32)
+                              * (0.5 ** np.arange(L, dtype=np.float32))[:, None, None])
+    want = rng.integers(0, K, size=(40, L)).astype(np.int32)
+    rec = oracle.decode(want, Cb, lib=lib).astype(np.float32)
+    got, _, _, _ = oracle.encode(rec, Cb, lib=lib)
+    assert np.array_equal(got, want), "round trip ids differ"
+
+
+def pin_decode_integer(lib):
+    rng = _rng(12)
+    L, K, D, M = 4, 50, 7, 300
+    C = rng.integers(-1000, 1000, size=(L, K, D)).astype(np.float32)
+    ids = rng.integers(0, K, size=(M, L)).astype(np.int32)
+    out = oracle.decode(ids, C, lib=lib)
+    Ci = C.astype(np.int64)
+    expect = np.zeros((M, D), np.int64)
+    for l in range(L):
+        expect += Ci[l][ids[:, l]]
+    assert np.array_equal(out, expect.astype(np.float64))
+    bad = ids.copy()
+    bad[5, 2] = K
+    try:
+        oracle.decode(bad, C, lib=lib)
+    except oracle.OracleError as e:
+        assert e.code == -5
+    else:
+        raise AssertionError("out-of-range id accepted")
+
+
+def load_golden():
+    C = {}
+    rows = []
+    with open(os.path.join(GOLDEN, "rvq_toy_2d.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("C "):
+                _, l, k, a, b = line.split()
+                C[(int(l), int(k))] = (float(a), float(b))
+            elif line.startswith("X "):
+                parts = [p.split() for p in line[2:].split("|")]
+                rows.append({"x": [float(v) for v in parts[0]],
+                             "ids": [int(v) for v in parts[1][1:]],
+                             "dist": [float(v) for v in parts[2][1:]],
+                             "residual": [float(v) for v in parts[3][1:]],
+                             "recon": [float(v) for v in parts[4][1:]]})
+    L = 1 + max(l for l, _ in C)
+    K = 1 + max(k for _, k in C)
+    cb = np.zeros((L, K, 2), np.float32)
+    for (l, k), v in C.items():
+        cb[l, k] = v
+    return cb, rows
+
+
+def pin_golden(lib):
+    cb, rows = load_golden()
+    x = np.array([r["x"] for r in rows], np.float32)
+    ids, res, rec, dist = oracle.encode(x, cb, lib=lib)
+    assert ids.tolist() == [r["ids"] for r in rows]
+    assert dist.tolist() == [r["dist"] for r in rows]
+    assert res.tolist() == [r["residual"] for r in rows]
+    assert rec.tolist() == [r["recon"] for r in rows]
+    assert oracle.decode(ids, cb, lib=lib).tolist() == [r["recon"] for r in rows]
+
+
+def pin_check_path(lib):
+    rng = _rng(13)
+    L, K, D, N = 3, 6, 4, 20
+    C = rng.standard_normal((L, K, D)).astype(np.float32)
+    x = rng.standard_normal((N, D)).astype(np.float32)
+    ids = rng.integers(0, K, size=(N, L)).astype(np.int32)       # an arbitrary path
+    rows = np.arange(N)
+    out = oracle.check_path(x, C, rows, ids, lib=lib)
+    for n in range(N):
+        r = x[n].astype(np.float64)
+        for l in range(L):
+            d = ((r[None, :] - C[l].astype(np.float64)) ** 2).sum(1)
+            a = int(np.argmin(d))
+            assert out["argmin"][n, l] == a
+            assert np.isclose(out["best"][n, l], d[a], rtol=1e-13)
+            assert np.isclose(out["second"][n, l], np.min(np.delete(d, a)), rtol=1e-13)
+            assert np.isclose(out["chosen"][n, l], d[ids[n, l]], rtol=1e-13)
+            r = r - C[l, ids[n, l]]
+    # distances() is the level-0 distance vector
+    d0 = oracle.distances(x[0].astype(np.float64), C[0], lib=lib)
+    assert np.allclose(d0, cdist(x[:1].astype(np.float64), C[0].astype(np.float64), "sqeuclidean")[0],
+                       rtol=1e-13)
+
+
+ALL_PINS = [pin_bruteforce, pin_nearest_neighbour_L1, pin_single_codeword,
+            pin_codebook_equals_features, pin_ties_lowest_index, pin_invariants, pin_planted,
+            pin_decode_integer, pin_golden, pin_check_path]
