@@ -1,0 +1,149 @@
+/*
+ * rvq.h -- C ABI of librvq.so: residual vector quantization (RVQ) of visual
+ * features into multi-level discrete token ids, and the gather-sum decode back
+ * to feature space, on one NVIDIA B200 (sm_100a).
+ *
+ * Method.  The LongCat-2.5 technical blog ("Visual Primitive Modeling" ->
+ * "Discrete Native Resolution Vision Transformer") applies RVQ to native-
+ * resolution encoder features so that an image becomes a sequence of
+ * multi-level tokens; the Meituan LongCat-2.5 open-source article (section
+ * "02 Visual Coding and 3D") says the quantizer adds detail level by level;
+ * Figure 1 of the blog shows the ids being reconstructed by a de-tokenizer; and
+ * "Offline Visual Preprocessing" fixes the tokenizer so ids are precomputed once.
+ * The pages give no code, sizes or metric.  This library implements the plain
+ * reading of that description: greedy RVQ under squared Euclidean distance,
+ *
+ *     r_0 = x;  for l in 0..L-1:  id_l = argmin_k ||r_l - C_l[k]||^2  (lowest k on ties)
+ *                                 r_{l+1} = r_l - C_l[id_l]
+ *     decode(ids) = sum_l C_l[id_l]           (fp32 accumulation, ascending l)
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller, 16-byte aligned,
+ *     row-major and densely packed.  The library keeps no device memory between
+ *     calls except lazily created profiling events.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
+ *     asynchronously; the call returns after enqueueing.
+ *   - The return value is an rvq_status.  Argument errors are detected on the host
+ *     before anything is enqueued (nothing is written).  Errors found on the device
+ *     (an id out of range, a pipeline wait that timed out) are written to the
+ *     optional caller-owned device word `*status` (0 = ok); the first error wins.
+ *     Read it after synchronising the stream.
+ *   - Inputs must be finite.  Calls that overlap on the GPU must not share output or
+ *     workspace buffers.
+ */
+#ifndef RVQ_H_
+#define RVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RVQ_API __attribute__((visibility("default")))
+#else
+#define RVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage type of features / codebooks. */
+typedef enum { RVQ_F32 = 0, RVQ_BF16 = 1 } rvq_dtype;
+
+typedef enum {
+    RVQ_OK = 0,
+    RVQ_ERR_ARG = -1,          /* null pointer, negative size, misaligned pointer, bad offsets */
+    RVQ_ERR_UNSUPPORTED = -2,  /* shape outside the supported range (see each call) */
+    RVQ_ERR_WORKSPACE = -3,    /* workspace missing or smaller than rvq_encode_workspace_size */
+    RVQ_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed */
+    RVQ_ERR_ID_RANGE = -5,     /* decode met an id outside [0, K) (device-detected) */
+    RVQ_ERR_TIMEOUT = -6       /* an encode pipeline wait gave up (device-detected) */
+} rvq_status;
+
+/* Per-level codebook statistics written by rvq_build_norms, RVQ_LEVEL_STATS floats per level:
+ *   [0] max_k ||C_l[k]||            [1] max_k ||C_l[k] - bf16(C_l[k])||
+ *   [2] max_k ||bf16(C_l[k])||      [3] max_k fl32(||C_l[k]||^2)
+ * (each rounded upward).  rvq_encode uses them to bound the error of its bf16 tensor-core
+ * distances and so decide when a candidate list provably holds the nearest codeword. */
+#define RVQ_LEVEL_STATS 4
+
+/*
+ * rvq_build_norms -- one-off preparation of a fixed codebook set ("Offline Visual
+ * Preprocessing": the tokenizer is fixed, so this runs once per codebook set).
+ *   codebooks    [L, K, D] in cb_dtype
+ *   norms        [L, K] fp32 out: ||C_l[k]||^2, accumulated in fp64, rounded to nearest
+ *   level_stats  [L, RVQ_LEVEL_STATS] fp32 out (see above)
+ *   cb_operand   [L, K, D] bf16 out: round-to-nearest-even copy used as the tensor-core
+ *                operand.  Required when cb_dtype == RVQ_F32; ignored (may be NULL) for
+ *                RVQ_BF16, where the codebooks themselves are the operand.
+ * Supported: 1 <= L <= 64, 1 <= K < 2^31, 16 <= D <= 8192 with D % 16 == 0.
+ */
+RVQ_API int rvq_build_norms(const void *codebooks, int cb_dtype, int L, int K, int D,
+                    float *norms, float *level_stats, void *cb_operand, void *stream);
+
+/*
+ * rvq_encode_workspace_size -- bytes of device workspace rvq_encode needs for these
+ * sizes on the current device.  Writes *bytes; returns an rvq_status.
+ */
+RVQ_API int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t *bytes);
+
+/*
+ * rvq_encode -- greedy RVQ of N feature vectors (blog, "Discrete Native Resolution Vision
+ * Transformer"; article, "02 Visual Coding and 3D": detail added level by level).
+ *   features     [N, D] in f_dtype (native-resolution patch features; several images may be
+ *                packed back to back)
+ *   codebooks    [L, K, D] in cb_dtype; cb_operand = the bf16 copy from rvq_build_norms
+ *                (NULL when cb_dtype == RVQ_BF16)
+ *   norms, level_stats  from rvq_build_norms for these codebooks
+ *   offsets      optional [B+1] int64 image boundaries of the packed batch (offsets[0] = 0,
+ *                non-decreasing, offsets[B] = N); checked on the device, not used in the
+ *                arithmetic (every row is quantized independently).  NULL with B = 0 if absent.
+ *   ids          [N, L] int32 out
+ *   residual     optional [N, D] fp32 out: r_L (fp32 running residual)
+ *   recon        optional [N, D] fp32 out: sum_l C_l[ids_l], same arithmetic as rvq_decode
+ *   fallbacks    optional [L] int32 out: per level, rows whose candidate list could not be
+ *                certified and were resolved by an exact scan of all K codewords
+ *   workspace    >= rvq_encode_workspace_size bytes, 256-byte aligned
+ * Distances: bf16 tensor-core scores ||c||^2 - 2 r.c select up to 8 candidates per row, which
+ * are rescored exactly (fp64 accumulation of fp32 differences); a row whose candidates cannot
+ * be proven to contain the nearest codeword is rescanned exactly.  Ties go to the lowest id.
+ * Supported: N >= 0 (N = 0 is a no-op), N < 2^31, 1 <= L <= 64, 1 <= K < 2^31, 64 <= D <= 4096 with
+ * D % 64 == 0.
+ */
+RVQ_API int rvq_encode(const void *features, int f_dtype, int64_t N, int D,
+               const void *codebooks, int cb_dtype, const void *cb_operand,
+               const float *norms, const float *level_stats, int L, int K,
+               const int64_t *offsets, int64_t B,
+               int32_t *ids, float *residual, float *recon, int32_t *fallbacks,
+               void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
+
+/*
+ * rvq_decode -- gather-sum de-tokenizer input (blog, Figure 1): recon[n] = sum_l C_l[ids[n,l]],
+ * fp32 accumulation in ascending l.
+ *   ids      [N, L] int32;  codebooks [L, K, D] in cb_dtype;  recon [N, D] fp32 out
+ * An id outside [0, K) contributes nothing and sets *status = RVQ_ERR_ID_RANGE.
+ * Supported: N >= 0, 1 <= L <= 64, 1 <= K < 2^31, 4 <= D with D % 4 == 0.
+ */
+RVQ_API int rvq_decode(const int32_t *ids, int64_t N, int L, const void *codebooks, int cb_dtype,
+               int K, int D, float *recon, int32_t *status, void *stream);
+
+/* Human-readable name of an rvq_status value (static string). */
+RVQ_API const char *rvq_status_str(int status);
+
+/*
+ * Measurement hooks (no counterpart on the pages).
+ * rvq_launch_count: number of kernels this library has launched since it was loaded.
+ * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on
+ *   its stream (not for use inside stream capture); rvq_profile_enable(0) stops and clears.
+ * rvq_profile_read: synchronises on the recorded events and returns the number of distance-
+ *   GEMM launches and their summed device time in milliseconds since the last enable.
+ */
+RVQ_API int64_t rvq_launch_count(void);
+RVQ_API int rvq_profile_enable(int enable);
+RVQ_API int rvq_profile_read(int64_t *gemm_launches, double *gemm_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RVQ_H_ */

@@ -1,0 +1,848 @@
+// rvq_encode.cu -- greedy residual vector quantization on sm_100a.
+//
+// Method (LongCat-2.5 technical blog, "Visual Primitive Modeling" -> "Discrete Native
+// Resolution Vision Transformer": RVQ over native-resolution encoder features; Meituan
+// LongCat-2.5 open-source article, "02 Visual Coding and 3D": detail is added level by
+// level): for every level l, every row takes the codeword nearest (squared Euclidean, lowest
+// index on ties) to its running residual and subtracts it.
+//
+// Per level the engine runs three kernels on the caller's stream:
+//
+//  1. dist_topk_kernel (tensor cores).  Scores s = r~ . c~ for all (row, codeword) pairs as a
+//     dense bf16 GEMM [N,D] x [D,K] -> fp32, tile 128 rows x 256 codewords, operands moved by
+//     TMA into a 4-stage shared-memory ring (128B swizzle), tcgen05.mma issued by one thread
+//     into a double-buffered TMEM accumulator (2 x 256 columns).  Four epilogue warps read the
+//     accumulator with tcgen05.ld (one TMEM lane = one row per thread), form the approximate
+//     shifted distance d~ = ||c||^2 - 2 s and keep a sorted running top-8 per row.  The distance
+//     matrix never leaves the SM.  A persistent grid of G CTAs splits the (row tile, codeword
+//     tile) units into G contiguous ranges, so the grid is balanced for any N; a CTA writes one
+//     partial top-8 list per row tile it touched.
+//  2. rescore_kernel (one warp per row).  Merges the partial lists, bounds the bf16 error E of
+//     every d~ from per-row and per-level norms, rescans exactly (fp64 accumulation of fp32
+//     differences) every candidate within 2E of the best, and accepts the exact minimum when
+//     it is provably below every non-candidate (certificate: best - ||r||^2 < T - E, T = the
+//     smallest d~ that was not kept).  Accepted rows write their id and update r -= C_l[id]
+//     (fp32) and the bf16 operand copy for the next level.  Other rows are queued.
+//  3. fallback_kernel.  Queued rows get an exact scan of all K codewords (fp64 accumulation)
+//     and the same update.
+//
+// Error bound used by the certificate, per row and level (r fp32 residual, r~ = bf16(r),
+// c stored codeword, c~ = bf16(c), n = fl32(||c||^2), s~ = tensor-core r~.c~ with fp32
+// accumulation, gamma = (D+16) 2^-22):
+//   | (||r-c||^2 - ||r||^2) - d~ | <= 2^-22 Nmax + 2 (||r-r~|| Cmax + ||r~|| dCmax)
+//                                     + 2 gamma ||r~|| C~max + 2^-23 (Nmax + 2 ||r~|| C~max)
+// where Cmax, dCmax, C~max, Nmax are the per-level maxima of ||c||, ||c-c~||, ||c~||, n from
+// rvq_build_norms (Cauchy-Schwarz on the two rounding error vectors, worst-case summation error
+// of the fp32 accumulator, rounding of n and of the epilogue FMA), inflated by 1%.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "rvq_device.cuh"
+#include "rvq_host.h"
+
+namespace rvq {
+
+int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_dtype, int K, int D, float *recon,
+                  int32_t *status, cudaStream_t s);
+
+namespace enc {
+
+constexpr int BM = 128;       // rows per tile (TMEM lanes)
+constexpr int BN = 256;       // codewords per tile (UMMA N)
+constexpr int BK = 64;        // bf16 elements per k-block = one 128-byte swizzle row
+constexpr int UK = 16;        // K of one kind::f16 UMMA
+constexpr int NSTAGE = 4;
+constexpr int TOPK = 8;
+constexpr int MAX_CAND = 64;  // candidates the rescore warp can merge (2 per lane)
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int GEMM_THREADS = 192;  // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
+constexpr int SMEM_BARRIER_OFF = NSTAGE * STAGE_BYTES;
+constexpr int GEMM_SMEM = SMEM_BARRIER_OFF + 256 + 1024;  // + barriers + alignment slack
+
+__device__ __forceinline__ float inf_f() { return __int_as_float(0x7f800000); }
+__device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
+
+struct GemmArgs {
+  const float *norms;  // [K] of this level
+  int64_t N;
+  int K;
+  int D;
+  int64_t U;  // units = row tiles x codeword tiles
+  int Tc;     // codeword tiles
+  int G;      // CTAs
+  int maxs;   // partial-list slots per row tile
+  float2 *cand;
+  int32_t *status;
+};
+
+// CTA that owns unit u when U units are split into G contiguous ranges [cU/G, (c+1)U/G).
+__host__ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t U, int G) {
+  return static_cast<int>(((u + 1) * static_cast<int64_t>(G) - 1) / U);
+}
+
+__device__ __forceinline__ void topk_insert(float (&bd)[TOPK], int (&bi)[TOPK], float x, int ix) {
+#pragma unroll
+  for (int t = 0; t < TOPK; ++t) {
+    const bool sw = x < bd[t];
+    const float tb = bd[t];
+    const int ti = bi[t];
+    bd[t] = sw ? x : tb;
+    bi[t] = sw ? ix : ti;
+    x = sw ? tb : x;
+    ix = sw ? ti : ix;
+  }
+}
+
+// Write one row's partial top-8 list for row tile rt into this CTA's slot.
+__device__ __forceinline__ void flush_topk(const GemmArgs &a, int64_t rt, int row_in_tile, const float (&bd)[TOPK],
+                                           const int (&bi)[TOPK]) {
+  const int64_t n = rt * BM + row_in_tile;
+  if (n < a.N) {
+    const int slot = static_cast<int>(blockIdx.x) - cta_of_unit(rt * a.Tc, a.U, a.G);
+    float2 *out = a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK;
+#pragma unroll
+    for (int t = 0; t < TOPK; ++t) out[t] = make_float2(bd[t], __int_as_float(bi[t]));
+  }
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    dist_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SMEM_BARRIER_OFF);
+  uint64_t *empty = full + NSTAGE;
+  uint64_t *tfull = empty + NSTAGE;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *mma_done = tempty + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  volatile int *never = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.U / a.G;
+  const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * a.U / a.G;
+  const int KB = a.D / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], BM);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < u1 && ok; ++u) {
+        const int64_t rt = u / a.Tc;
+        const int ct = static_cast<int>(u - rt * a.Tc);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          uint8_t *sa = smem + s * STAGE_BYTES;
+          tma_load_2d(&tmA, &full[s], sa, kb * BK, static_cast<int32_t>(rt * BM));
+          tma_load_2d(&tmB, &full[s], sa + A_BYTES, kb * BK, ct * BN);
+          ++issued;
+          if (++s == NSTAGE) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(a.status, RVQ_ERR_TIMEOUT);
+        // no bulk copy may still be landing in shared memory when the block exits
+        const int64_t pending = issued < NSTAGE ? issued : NSTAGE;
+        for (int64_t j = 0; j < pending; ++j) {
+          int back = s - 1 - static_cast<int>(j);
+          uint32_t p = ph;
+          while (back < 0) {
+            back += NSTAGE;
+            p ^= 1u;
+          }
+          mbar_wait(&full[back], p, never);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t i = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < u1 && ok; ++u, ++i) {
+        const int buf = static_cast<int>(i & 1);
+        const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = sdesc_k128(sa);
+          const uint64_t bd = sdesc_k128(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            umma_f16(dt, ad + static_cast<uint64_t>(k * UK * 2 / 16), bd + static_cast<uint64_t>(k * UK * 2 / 16),
+                     idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+          if (++s == NSTAGE) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(a.status, RVQ_ERR_TIMEOUT);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: running top-8
+    const int row_in_tile = warp * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    const bool vec_norms = (a.K & 3) == 0;
+    float bd[TOPK];
+    int bi[TOPK];
+#pragma unroll
+    for (int t = 0; t < TOPK; ++t) {
+      bd[t] = inf_f();
+      bi[t] = -1;
+    }
+    int64_t cur_rt = -1;
+    int64_t i = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1; ++u, ++i) {
+      const int64_t rt = u / a.Tc;
+      const int ct = static_cast<int>(u - rt * a.Tc);
+      if (rt != cur_rt) {
+        if (cur_rt >= 0) flush_topk(a, cur_rt, row_in_tile, bd, bi);
+#pragma unroll
+        for (int t = 0; t < TOPK; ++t) {
+          bd[t] = inf_f();
+          bi[t] = -1;
+        }
+        cur_rt = rt;
+      }
+      const int buf = static_cast<int>(i & 1);
+      const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
+      const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int col0 = ct * BN;
+      const int nvalid = min(BN, a.K - col0);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld_32x32(lane_base + static_cast<uint32_t>(buf * BN + ch * 32), v);
+        tmem_ld_wait();
+        if (ch == BN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&tempty[buf]);
+        }
+        const int c0 = col0 + ch * 32;
+        float d[32];
+        if (ch * 32 + 32 <= nvalid && vec_norms) {
+          const float4 *np = reinterpret_cast<const float4 *>(a.norms + c0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 nn = __ldg(np + j);
+            d[4 * j + 0] = fmaf(-2.f, __uint_as_float(v[4 * j + 0]), nn.x);
+            d[4 * j + 1] = fmaf(-2.f, __uint_as_float(v[4 * j + 1]), nn.y);
+            d[4 * j + 2] = fmaf(-2.f, __uint_as_float(v[4 * j + 2]), nn.z);
+            d[4 * j + 3] = fmaf(-2.f, __uint_as_float(v[4 * j + 3]), nn.w);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            d[j] = (ch * 32 + j < nvalid) ? fmaf(-2.f, __uint_as_float(v[j]), __ldg(a.norms + c0 + j)) : inf_f();
+        }
+        float m = d[0];
+#pragma unroll
+        for (int j = 1; j < 32; ++j) m = fminf(m, d[j]);
+        if (__any_sync(0xffffffffu, m < bd[TOPK - 1])) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (__any_sync(0xffffffffu, d[j] < bd[TOPK - 1])) topk_insert(bd, bi, d[j], c0 + j);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(a.status, RVQ_ERR_TIMEOUT);
+    } else if (cur_rt >= 0) {
+      flush_topk(a, cur_rt, row_in_tile, bd, bi);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- row kernels
+
+template <bool BF16>
+__device__ __forceinline__ float4 ld4(const void *p, int64_t off) {
+  if constexpr (BF16) {
+    uint2 raw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p) + off));
+    float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
+    float2 y = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
+    return make_float4(x.x, x.y, y.x, y.y);
+  } else {
+    return __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off));
+  }
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_min_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16 *p, float4 v, float4 *rounded) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t *>(&a);
+  packed.y = *reinterpret_cast<uint32_t *>(&b);
+  *reinterpret_cast<uint2 *>(p) = packed;
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  *rounded = make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// r (fp32) -> bf16 operand row + (||r - r~||, ||r~||); one warp per row, lanes stride by 4.
+__device__ __forceinline__ float2 write_operand_row(const float *r, __nv_bfloat16 *rt, int D, int lane) {
+  float e2 = 0.f, q2 = 0.f;
+  for (int i = lane * 4; i < D; i += 128) {
+    const float4 v = *reinterpret_cast<const float4 *>(r + i);
+    float4 q;
+    store_bf16x4(rt + i, v, &q);
+    const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+    e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+    q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+  }
+  e2 = warp_sum_f(e2);
+  q2 = warp_sum_f(q2);
+  return make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
+}
+
+// r_0 = fp32(x), its bf16 operand copy and row statistics; also clears the fallback counters
+// and checks the packed-batch offsets.
+template <bool X_BF16>
+__global__ void __launch_bounds__(256) init_kernel(const void *__restrict__ x, int64_t N, int D, float *__restrict__ R,
+                                                   __nv_bfloat16 *__restrict__ Rt, float2 *__restrict__ rowstat,
+                                                   int32_t *__restrict__ fb_count, int L,
+                                                   const int64_t *__restrict__ offsets, int64_t B,
+                                                   int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gtid < L) fb_count[gtid] = 0;
+  if (offsets) {
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t b = gtid; b < B; b += nthreads)
+      if (offsets[b] > offsets[b + 1]) set_status(status, RVQ_ERR_ARG);
+    if (gtid == 0 && (offsets[0] != 0 || offsets[B] != N)) set_status(status, RVQ_ERR_ARG);
+  }
+  const int64_t n = gtid >> 5;
+  if (n >= N) return;
+  float *r = R + n * D;
+  for (int i = lane * 4; i < D; i += 128) {
+    const float4 v = ld4<X_BF16>(x, n * D + i);
+    *reinterpret_cast<float4 *>(r + i) = v;
+  }
+  __syncwarp();
+  const float2 st = write_operand_row(r, Rt + n * D, D, lane);
+  if (lane == 0) rowstat[n] = st;
+}
+
+struct RowArgs {
+  int64_t N;
+  int D, K, L, l;
+  int Tc, G, maxs;
+  int64_t U;
+  const float2 *cand;
+  float2 *rowstat;
+  float *R;
+  __nv_bfloat16 *Rt;
+  const void *cb;        // stored codebooks [L,K,D]
+  const float *stats;    // this level's RVQ_LEVEL_STATS floats
+  int32_t *ids;
+  int32_t *fb_list;
+  int32_t *fb_count;     // this level's counter
+  int32_t *status;
+  int last;              // no operand copy needed after the last level
+};
+
+__device__ __forceinline__ float error_bound(const float *st, float2 rs, int D) {
+  const float cmax = st[0], dcmax = st[1], cqmax = st[2], nmax = st[3];
+  const float gamma = static_cast<float>(D + 16) * 2.384185791015625e-07f;  // 2^-22
+  const float e = 2.384185791015625e-07f * nmax + 2.f * (rs.x * cmax + rs.y * dcmax) +
+                  2.f * gamma * rs.y * cqmax + 1.1920928955078125e-07f * (nmax + 2.f * rs.y * cqmax);
+  return 1.01f * e;
+}
+
+// Exact squared distance ||r - c||^2 with fp32 differences widened to fp64 and fp64 sums.
+template <bool CB_BF16>
+__device__ __forceinline__ double exact_dist(const float *r, const void *cb, int64_t coff, int D, int lane) {
+  double s = 0.0;
+  for (int i = lane * 4; i < D; i += 128) {
+    const float4 v = *reinterpret_cast<const float4 *>(r + i);
+    const float4 c = ld4<CB_BF16>(cb, coff + i);
+    const double a = static_cast<double>(v.x) - c.x, b = static_cast<double>(v.y) - c.y;
+    const double e = static_cast<double>(v.z) - c.z, f = static_cast<double>(v.w) - c.w;
+    s += a * a + b * b + e * e + f * f;
+  }
+  return warp_sum_d(s);
+}
+
+// r -= c (fp32), write the ids entry and, unless this was the last level, the next operand row.
+template <bool CB_BF16>
+__device__ __forceinline__ void accept_row(const RowArgs &a, int64_t n, int id, int lane) {
+  float *r = a.R + n * a.D;
+  const int64_t coff = (static_cast<int64_t>(a.l) * a.K + id) * a.D;
+  for (int i = lane * 4; i < a.D; i += 128) {
+    float4 v = *reinterpret_cast<float4 *>(r + i);
+    const float4 c = ld4<CB_BF16>(a.cb, coff + i);
+    v.x -= c.x;
+    v.y -= c.y;
+    v.z -= c.z;
+    v.w -= c.w;
+    *reinterpret_cast<float4 *>(r + i) = v;
+  }
+  __syncwarp();
+  if (!a.last) {
+    const float2 st = write_operand_row(r, a.Rt + n * a.D, a.D, lane);
+    if (lane == 0) a.rowstat[n] = st;
+  }
+  if (lane == 0) a.ids[n * a.L + a.l] = id;
+}
+
+template <bool CB_BF16>
+__global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (n >= a.N) return;
+  const int64_t rt = n / BM;
+  const int rin = static_cast<int>(n - rt * BM);
+  const int c0 = cta_of_unit(rt * a.Tc, a.U, a.G);
+  const int c1 = cta_of_unit(rt * a.Tc + a.Tc - 1, a.U, a.G);
+  const int ncand = (c1 - c0 + 1) * TOPK;
+
+  float dv[2];
+  int iv[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = lane + 32 * h;
+    dv[h] = inf_f();
+    iv[h] = -1;
+    if (e < ncand) {
+      const int slot = e / TOPK, t = e - slot * TOPK;
+      const float2 c = a.cand[((rt * a.maxs + slot) * BM + rin) * TOPK + t];
+      dv[h] = c.x;
+      iv[h] = __float_as_int(c.y);
+    }
+  }
+  // T: smallest score that some list dropped (a list's last entry; +inf if the list is short)
+  float tl = inf_f();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = lane + 32 * h;
+    if (e < ncand && (e % TOPK) == TOPK - 1) tl = fminf(tl, dv[h]);
+  }
+  const float T = warp_min_f(tl);
+  const float dmin = warp_min_f(fminf(dv[0], dv[1]));
+  const float E = error_bound(a.stats, a.rowstat[n], a.D);
+
+  const float *r = a.R + n * a.D;
+  double rr = 0.0;
+  for (int i = lane * 4; i < a.D; i += 128) {
+    const float4 v = *reinterpret_cast<const float4 *>(r + i);
+    rr += static_cast<double>(v.x) * v.x + static_cast<double>(v.y) * v.y + static_cast<double>(v.z) * v.z +
+          static_cast<double>(v.w) * v.w;
+  }
+  rr = warp_sum_d(rr);
+
+  double best = inf_d();
+  int best_id = 0x7fffffff;
+  const float lim = dmin + 2.f * E;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    unsigned mask = __ballot_sync(0xffffffffu, iv[h] >= 0 && dv[h] <= lim);
+    while (mask) {
+      const int src = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const int id = __shfl_sync(0xffffffffu, iv[h], src);
+      const double d = exact_dist<CB_BF16>(r, a.cb, (static_cast<int64_t>(a.l) * a.K + id) * a.D, a.D, lane);
+      if (d < best || (d == best && id < best_id)) {
+        best = d;
+        best_id = id;
+      }
+    }
+  }
+  const bool certified = best_id != 0x7fffffff && (best - rr) < (static_cast<double>(T) - static_cast<double>(E));
+  if (!certified) {
+    if (lane == 0) {
+      const int pos = atomicAdd(a.fb_count, 1);
+      a.fb_list[pos] = static_cast<int32_t>(n);
+    }
+    return;
+  }
+  accept_row<CB_BF16>(a, n, best_id, lane);
+}
+
+// Exact scan of all K codewords for the queued rows of this level.
+template <bool CB_BF16>
+__global__ void __launch_bounds__(256) fallback_kernel(const RowArgs a) {
+  extern __shared__ double sr[];  // residual row widened to fp64
+  __shared__ double wbest[8];
+  __shared__ int wid[8];
+  __shared__ int chosen;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int count = *a.fb_count;
+  for (int j = blockIdx.x; j < count; j += gridDim.x) {
+    const int64_t n = a.fb_list[j];
+    const float *r = a.R + n * a.D;
+    __syncthreads();
+    for (int i = threadIdx.x; i < a.D; i += blockDim.x) sr[i] = static_cast<double>(r[i]);
+    __syncthreads();
+    double bd = inf_d();
+    int bk = 0x7fffffff;
+    for (int k = warp; k < a.K; k += 8) {
+      const int64_t coff = (static_cast<int64_t>(a.l) * a.K + k) * a.D;
+      double s = 0.0;
+      if constexpr (CB_BF16) {
+        const __nv_bfloat16 *c = static_cast<const __nv_bfloat16 *>(a.cb) + coff;
+        for (int i = lane; i < a.D; i += 32) {
+          const double t = sr[i] - static_cast<double>(__bfloat162float(c[i]));
+          s += t * t;
+        }
+      } else {
+        const float *c = static_cast<const float *>(a.cb) + coff;
+        for (int i = lane; i < a.D; i += 32) {
+          const double t = sr[i] - static_cast<double>(__ldg(c + i));
+          s += t * t;
+        }
+      }
+      s = warp_sum_d(s);
+      if (s < bd) {
+        bd = s;
+        bk = k;
+      }
+    }
+    if (lane == 0) {
+      wbest[warp] = bd;
+      wid[warp] = bk;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double b = wbest[0];
+      int k = wid[0];
+      for (int w = 1; w < 8; ++w)
+        if (wbest[w] < b || (wbest[w] == b && wid[w] < k)) {
+          b = wbest[w];
+          k = wid[w];
+        }
+      chosen = k;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      if (chosen >= 0 && chosen < a.K) {
+        accept_row<CB_BF16>(a, n, chosen, lane);
+      } else if (lane == 0) {  // only reachable with non-finite inputs
+        a.ids[n * a.L + a.l] = -1;
+        set_status(a.status, RVQ_ERR_ARG);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host plan
+
+struct Plan {
+  int64_t RT;
+  int Tc;
+  int64_t U;
+  int G;
+  int maxs;
+};
+
+inline Plan make_plan(int64_t N, int K, int sms) {
+  Plan p;
+  p.RT = (N + BM - 1) / BM;
+  p.Tc = (K + BN - 1) / BN;
+  p.U = p.RT * p.Tc;
+  // every CTA covers at least f = floor(U/G) units, so a row tile (Tc consecutive units) meets
+  // at most 1 + ceil((Tc-1)/f) CTAs; keep that within the rescore warp's candidate capacity
+  const int64_t slots_cap = MAX_CAND / TOPK;
+  const int64_t need_f = std::max<int64_t>(1, (p.Tc - 1 + slots_cap - 2) / (slots_cap - 1));
+  int64_t G = std::min<int64_t>(sms, p.U);
+  G = std::min<int64_t>(G, std::max<int64_t>(1, p.U / need_f));
+  p.G = static_cast<int>(G);
+  const int64_t f = p.U / p.G;
+  p.maxs = static_cast<int>(std::min<int64_t>(p.G, 1 + (p.Tc - 1 + f - 1) / f));
+  return p;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+  size_t R, Rt, rowstat, cand, fb_list, fb_count, total;
+};
+
+inline Layout make_layout(int64_t N, int D, const Plan &p) {
+  Layout w;
+  size_t off = 0;
+  w.R = off;
+  off += align256(static_cast<size_t>(N) * D * 4);
+  w.Rt = off;
+  off += align256(static_cast<size_t>(N) * D * 2);
+  w.rowstat = off;
+  off += align256(static_cast<size_t>(N) * 8);
+  w.cand = off;
+  off += align256(static_cast<size_t>(p.RT) * p.maxs * BM * TOPK * 8);
+  w.fb_list = off;
+  off += align256(static_cast<size_t>(N) * 4);
+  w.fb_count = off;
+  off += align256(64 * 4);
+  w.total = off;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 [rows, D] row-major, box = BK elements x box_rows rows, 128B swizzle, zero fill outside.
+inline bool make_map(CUtensorMap *m, const void *base, int64_t rows, int D, int box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace enc
+}  // namespace rvq
+
+extern "C" int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t *bytes) {
+  using namespace rvq;
+  if (!bytes || N < 0 || D < 1 || L < 1 || K < 1) return RVQ_ERR_ARG;
+  if (L > 64 || D < 64 || D > 4096 || D % 64 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  int sms = 0;
+  int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, sms);
+  *bytes = enc::make_layout(N, D, p).total;
+  return RVQ_OK;
+}
+
+extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, const void *codebooks, int cb_dtype,
+                          const void *cb_operand, const float *norms, const float *level_stats, int L, int K,
+                          const int64_t *offsets, int64_t B, int32_t *ids, float *residual, float *recon,
+                          int32_t *fallbacks, void *workspace, size_t workspace_bytes, int32_t *status,
+                          void *stream) {
+  using namespace rvq;
+  using namespace rvq::enc;
+  if (N < 0 || D < 1 || L < 1 || K < 1 || B < 0) return RVQ_ERR_ARG;
+  if ((f_dtype != RVQ_F32 && f_dtype != RVQ_BF16) || (cb_dtype != RVQ_F32 && cb_dtype != RVQ_BF16))
+    return RVQ_ERR_ARG;
+  if (L > 64 || D < 64 || D > 4096 || D % 64 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  if (offsets == nullptr && B != 0) return RVQ_ERR_ARG;
+  if (N == 0) return RVQ_OK;
+  if (!features || !codebooks || !norms || !level_stats || !ids) return RVQ_ERR_ARG;
+  if (cb_dtype == RVQ_F32 && !cb_operand) return RVQ_ERR_ARG;
+  const void *op = cb_dtype == RVQ_BF16 ? codebooks : cb_operand;
+  if (!aligned16(features) || !aligned16(codebooks) || !aligned16(op) || !aligned16(norms) ||
+      (residual && !aligned16(residual)) || (recon && !aligned16(recon)) || (reinterpret_cast<uintptr_t>(ids) & 3u))
+    return RVQ_ERR_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RVQ_ERR_WORKSPACE;
+  int sms = 0;
+  int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const Plan p = make_plan(N, K, sms);
+  const Layout w = make_layout(N, D, p);
+  if (workspace_bytes < w.total) return RVQ_ERR_WORKSPACE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *R = residual ? residual : reinterpret_cast<float *>(ws + w.R);
+  __nv_bfloat16 *Rt = reinterpret_cast<__nv_bfloat16 *>(ws + w.Rt);
+  float2 *rowstat = reinterpret_cast<float2 *>(ws + w.rowstat);
+  float2 *cand = reinterpret_cast<float2 *>(ws + w.cand);
+  int32_t *fb_list = reinterpret_cast<int32_t *>(ws + w.fb_list);
+  int32_t *fb_count = reinterpret_cast<int32_t *>(ws + w.fb_count);
+
+  CUtensorMap tmA;
+  if (!make_map(&tmA, Rt, N, D, BM)) return RVQ_ERR_CUDA;
+
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(dist_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM) !=
+        cudaSuccess)
+      return RVQ_ERR_CUDA;
+    attr_done = true;
+  }
+
+  {
+    const int64_t threads = N * 32;
+    const int64_t blocks = (threads + 255) / 256;
+    if (f_dtype == RVQ_BF16)
+      init_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(features, N, D, R, Rt, rowstat, fb_count, L,
+                                                                       offsets, B, status);
+    else
+      init_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(features, N, D, R, Rt, rowstat, fb_count, L,
+                                                                        offsets, B, status);
+    note_launch();
+    if ((st = check_launch()) != RVQ_OK) return st;
+  }
+
+  const int64_t row_blocks = (N * 32 + 255) / 256;
+  const int fb_blocks = 2 * sms;
+  const size_t fb_smem = static_cast<size_t>(D) * sizeof(double);
+  for (int l = 0; l < L; ++l) {
+    const size_t lvl = static_cast<size_t>(l) * K * D * 2;
+    CUtensorMap tmB;
+    if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, BN)) return RVQ_ERR_CUDA;
+    GemmArgs ga;
+    ga.norms = norms + static_cast<size_t>(l) * K;
+    ga.N = N;
+    ga.K = K;
+    ga.D = D;
+    ga.U = p.U;
+    ga.Tc = p.Tc;
+    ga.G = p.G;
+    ga.maxs = p.maxs;
+    ga.cand = cand;
+    ga.status = status;
+    profile_begin(s);
+    dist_topk_kernel<<<p.G, GEMM_THREADS, GEMM_SMEM, s>>>(tmA, tmB, ga);
+    profile_end(s);
+    note_launch();
+    if ((st = check_launch()) != RVQ_OK) return st;
+
+    RowArgs ra;
+    ra.N = N;
+    ra.D = D;
+    ra.K = K;
+    ra.L = L;
+    ra.l = l;
+    ra.Tc = p.Tc;
+    ra.G = p.G;
+    ra.maxs = p.maxs;
+    ra.U = p.U;
+    ra.cand = cand;
+    ra.rowstat = rowstat;
+    ra.R = R;
+    ra.Rt = Rt;
+    ra.cb = codebooks;
+    ra.stats = level_stats + static_cast<size_t>(l) * RVQ_LEVEL_STATS;
+    ra.ids = ids;
+    ra.fb_list = fb_list;
+    ra.fb_count = fb_count + l;
+    ra.status = status;
+    ra.last = l == L - 1;
+    if (cb_dtype == RVQ_BF16) {
+      rescore_kernel<true><<<static_cast<unsigned>(row_blocks), 256, 0, s>>>(ra);
+      fallback_kernel<true><<<fb_blocks, 256, fb_smem, s>>>(ra);
+    } else {
+      rescore_kernel<false><<<static_cast<unsigned>(row_blocks), 256, 0, s>>>(ra);
+      fallback_kernel<false><<<fb_blocks, 256, fb_smem, s>>>(ra);
+    }
+    note_launch(2);
+    if ((st = check_launch()) != RVQ_OK) return st;
+  }
+  if (fallbacks) {
+    if (cudaMemcpyAsync(fallbacks, fb_count, sizeof(int32_t) * L, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return RVQ_ERR_CUDA;
+  }
+  if (recon) {
+    st = launch_decode(ids, N, L, codebooks, cb_dtype, K, D, recon, status, s);
+    if (st != RVQ_OK) return st;
+  }
+  return RVQ_OK;
+}

@@ -1,0 +1,241 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Small workloads are compared on every row; the large ones on seeded row samples (first and
+last rows and image boundaries included) plus properties checked on every row.  The id rule
+and tolerances are in tests/parity.py.
+"""
+import numpy as np
+import pytest
+
+import workloads
+from tests import parity
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU hosts, run only with a GPU
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import multimodal_visual_tokenization_b200 as mvt  # noqa: E402
+
+
+def dev(a, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    return t.cuda()
+
+
+def run_encode(x, C, f_dtype="f32", cb_dtype="f32", offsets=None):
+    tok = mvt.Tokenizer(dev(C, cb_dtype))
+    fb = torch.zeros(C.shape[0], dtype=torch.int32, device="cuda")
+    off = None if offsets is None else torch.from_numpy(offsets).cuda()
+    ids, res, rec = tok.encode(dev(x, f_dtype), offsets=off, residual=True, recon=True, fallbacks=fb)
+    torch.cuda.synchronize()
+    return tok, ids.cpu().numpy(), res.cpu().numpy(), rec.cpu().numpy(), fb.cpu().numpy()
+
+
+def full_check(x, C, ids, res, rec, rows=None):
+    rows = np.arange(x.shape[0]) if rows is None else rows
+    rep = parity.check_ids(x, C, rows, ids)
+    rep.update(parity.check_recon(x, C, rows, ids, rec, res))
+    parity.check_all_rows(x, ids, C.shape[1], rec, res)
+    return rep
+
+
+def test_tiny_all_rows():
+    g = workloads.generate("tiny")
+    _, ids, res, rec, fb = run_encode(g["x"], g["codebooks"])
+    rep = full_check(g["x"], g["codebooks"], ids, res, rec)
+    assert rep["exact"] == rep["row_levels"]
+    assert (ids[:, 0] == g["planted"][:, 0]).all()
+
+
+def test_image_sampled():
+    g = workloads.generate("image")
+    x, C = g["x"], g["codebooks"]
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    rows = workloads.sample_rows(len(x), 192, seed=1)
+    rep = full_check(x, C, ids, res, rec, rows)
+    print("image", rep, "fallbacks", fb.tolist())
+    assert (ids[:, 0] == g["planted"][:, 0]).all()         # planted level 0, every row
+
+
+def test_image_small_all_rows():
+    g = workloads.generate("image", n_override=300)
+    x, C = g["x"], g["codebooks"]
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    rep = full_check(x, C, ids, res, rec)
+    assert rep["rows_equal_free_running"] == rep["rows"]
+
+
+def test_packed_sampled():
+    g = workloads.generate("packed")
+    x, C, off = g["x"], g["codebooks"], g["offsets"]
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32", offsets=off)
+    rows = workloads.sample_rows(len(x), 24, seed=2, offsets=off[::8])
+    rep = full_check(x, C, ids, res, rec, rows)
+    print("packed", rep, "fallbacks", fb.tolist())
+    assert (ids[:, 0] == g["planted"][:, 0]).all()
+
+
+def test_offline_sampled():
+    g = workloads.generate("offline")
+    x, C = g["x"], g["codebooks"]
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    rows = workloads.sample_rows(len(x), 96, seed=3)
+    rep = full_check(x, C, ids, res, rec, rows)
+    print("offline", rep, "fallbacks", fb.tolist())
+    assert (ids[:, 0] == g["planted"][:, 0]).mean() > 0.999   # mixture centre recovered
+
+
+def test_detok_decode_and_round_trip():
+    g = workloads.generate("detok")
+    C, want = g["codebooks"], g["planted"]
+    tok = mvt.Tokenizer(dev(C, "bf16"))
+    ids_d = torch.from_numpy(want).cuda()
+    rec = tok.decode(ids_d)
+    torch.cuda.synchronize()
+    rec_h = rec.cpu().numpy()
+    rows = workloads.sample_rows(len(want), 4096, seed=4)
+    parity.check_recon(None, C, rows, want, recon_gpu=rec_h)
+    # re-encode the fp32 reconstruction: the planted ids must come back on every row
+    fb = torch.zeros(C.shape[0], dtype=torch.int32, device="cuda")
+    ids, res, rec2 = tok.encode(rec, residual=True, recon=True, fallbacks=fb)
+    torch.cuda.synchronize()
+    ids_h = ids.cpu().numpy()
+    assert np.array_equal(ids_h, want), f"{int((ids_h != want).any(1).sum())} rows differ"
+    srows = workloads.sample_rows(len(want), 12, seed=5)
+    parity.check_ids(rec_h, C, srows, ids_h)
+    parity.check_recon(rec_h, C, srows, ids_h, rec2.cpu().numpy(), res.cpu().numpy())
+
+
+EDGE = [
+    # N, D, L, K, f_dtype, cb_dtype
+    (1, 64, 2, 16, "f32", "f32"),
+    (127, 64, 3, 300, "f32", "f32"),
+    (129, 128, 2, 257, "bf16", "f32"),
+    (300, 256, 2, 1, "f32", "f32"),
+    (513, 1024, 2, 512, "bf16", "bf16"),
+    (200, 64, 4, 4096, "f32", "bf16"),
+    (1000, 192, 3, 1000, "bf16", "f32"),
+    (4100, 64, 2, 33, "f32", "f32"),
+]
+
+
+@pytest.mark.parametrize("N,D,L,K,fd,cd", EDGE)
+def test_edge_shapes(N, D, L, K, fd, cd):
+    rng = np.random.Generator(np.random.PCG64([N, D, L, K]))
+    C = rng.standard_normal((L, K, D)).astype(np.float32) * (0.5 ** np.arange(L, dtype=np.float32))[:, None, None]
+    x = rng.standard_normal((N, D)).astype(np.float32)
+    if cd == "bf16":
+        C = workloads.round_bf16(C)
+    if fd == "bf16":
+        x = workloads.round_bf16(x)
+    _, ids, res, rec, fb = run_encode(x, C, fd, cd)
+    full_check(x, C, ids, res, rec)
+
+
+def test_duplicate_and_zero_codebooks():
+    rng = np.random.Generator(np.random.PCG64(21))
+    base = rng.standard_normal((40, 64)).astype(np.float32)
+    C = np.stack([np.concatenate([base, base, base]), np.zeros((120, 64), np.float32)])
+    x = rng.standard_normal((500, 64)).astype(np.float32)
+    _, ids, res, rec, fb = run_encode(x, C)
+    assert (ids[:, 0] < 40).all(), "duplicate codewords must resolve to the lowest index"
+    assert (ids[:, 1] == 0).all(), "all-zero level must pick codeword 0"
+    full_check(x, C, ids, res, rec)
+
+
+def test_codebook_equals_features():
+    rng = np.random.Generator(np.random.PCG64(22))
+    x = rng.standard_normal((600, 128)).astype(np.float32)
+    perm = rng.permutation(600)
+    C = x[perm][None]
+    _, ids, res, rec, fb = run_encode(x, C)
+    assert np.array_equal(ids[:, 0], np.argsort(perm))
+    assert np.abs(res).max() == 0.0
+
+
+@pytest.mark.parametrize("copies", [2, 16])
+def test_near_ties_use_exact_rescoring(copies):
+    """Groups of codewords 1e-7..1e-4 apart (relative): bf16 scores cannot order them.  Pairs
+    must be settled by exact rescoring of the candidate list; groups of 16 overflow the top-8
+    list, fail the certificate and must be settled by the exact full scan."""
+    rng = np.random.Generator(np.random.PCG64(23 + copies))
+    D, G, N = 256, 32, 400
+    base = rng.standard_normal((G, D)).astype(np.float32)
+    eps = (10.0 ** rng.uniform(-7, -4, size=(copies, G, 1))).astype(np.float32)
+    eps[0] = 0.0
+    C = (base[None] * (1 + eps)).reshape(1, copies * G, D)
+    pick = rng.integers(0, G, size=N)
+    x = base[pick] + 1e-3 * rng.standard_normal((N, D)).astype(np.float32)
+    _, ids, res, rec, fb = run_encode(x, C)
+    rep = full_check(x, C, ids, res, rec)
+    print("near ties", copies, rep, "fallbacks", fb.tolist())
+    if copies > 8:
+        assert fb.sum() > 0
+
+
+def test_decode_out_of_range_sets_status():
+    C = np.random.Generator(np.random.PCG64(24)).standard_normal((2, 10, 64)).astype(np.float32)
+    tok = mvt.Tokenizer(dev(C, "f32"))
+    ids = torch.zeros((5, 2), dtype=torch.int32, device="cuda")
+    ids[3, 1] = 10
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rec = tok.decode(ids, status=st, check=False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == -5
+    want = np.array(C[0, 0] + C[1, 0], np.float32)
+    assert np.allclose(rec[0].cpu().numpy(), want)
+    assert np.allclose(rec[3].cpu().numpy(), C[0, 0])      # bad level contributes nothing
+
+
+def test_bad_offsets_set_status():
+    rng = np.random.Generator(np.random.PCG64(25))
+    C = rng.standard_normal((1, 32, 64)).astype(np.float32)
+    x = rng.standard_normal((50, 64)).astype(np.float32)
+    tok = mvt.Tokenizer(dev(C, "f32"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    off = torch.tensor([0, 30, 20, 50], dtype=torch.int64, device="cuda")
+    tok.encode(dev(x, "f32"), offsets=off, status=st, check=False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == -1
+
+
+def test_empty_batch_is_noop():
+    C = np.random.Generator(np.random.PCG64(26)).standard_normal((2, 16, 64)).astype(np.float32)
+    tok = mvt.Tokenizer(dev(C, "f32"))
+    ids, _, _ = tok.encode(torch.empty((0, 64), device="cuda"))
+    assert ids.shape == (0, 2)
+
+
+def test_norms_and_stats():
+    g = workloads.generate("image", n_override=8)
+    C = g["codebooks"]
+    tok = mvt.Tokenizer(dev(C, "f32"))
+    torch.cuda.synchronize()
+    n = tok.norms.cpu().numpy().astype(np.float64)
+    want = (C.astype(np.float64) ** 2).sum(-1)
+    assert np.allclose(n, want, rtol=2 ** -23, atol=0)
+    op = tok.operand.float().cpu().numpy()
+    assert np.array_equal(op, workloads.round_bf16(C))
+    st = tok.level_stats.cpu().numpy()
+    cn = np.sqrt(want).max(1)
+    assert (st[:, 0] >= cn * (1 - 1e-6)).all() and (st[:, 0] <= cn * (1 + 1e-5)).all()
+    assert (st[:, 3] >= want.max(1) * (1 - 1e-6)).all()
+    err = np.sqrt(((C.astype(np.float64) - op) ** 2).sum(-1)).max(1)
+    assert (st[:, 1] >= err * (1 - 1e-5)).all() and (st[:, 1] <= err * (1 + 1e-4)).all()
+
+
+def test_launch_count_and_profile_hooks():
+    g = workloads.generate("tiny")
+    tok = mvt.Tokenizer(dev(g["codebooks"], "f32"))
+    x = dev(g["x"], "f32")
+    before = mvt.rvq_launch_count()
+    assert mvt.rvq_profile_enable(True) == 0
+    tok.encode(x)
+    code, n, ms = mvt.rvq_profile_read()
+    mvt.rvq_profile_enable(False)
+    assert code == 0 and n == g["spec"].L and ms > 0
+    assert mvt.rvq_launch_count() - before == 1 + 3 * g["spec"].L
