@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Throughput of the RVQ visual-tokenization hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic native-resolution
+patch features, through the C ABI:
+    rvq_build_norms (codeword norms + bf16 operand copy)
+    rvq_encode      (greedy RVQ: ids, fp32 residual and recon)
+    rvq_decode      (gather-sum of the produced ids)
+Metric: tokens (feature vectors) per second, in millions.  `value` is measured with the
+inputs resident in HBM; `e2e` repeats it through the same calls with the features copied
+from pinned host memory every step and the ids + decoded recon copied back.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload image] [--impl reference]
+Multi-GPU: launched by torchrun, one rank per GPU; every rank quantizes its own batch
+(weak scaling, no data-path collective); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "RVQ encode Mtokens/s (L levels, K codes, dim D) and % tensor-core peak; decode GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 512 << 20          # > 126 MB L2
+GEMM_KERNEL_SRC = os.path.join(ROOT, "multimodal_visual_tokenization_b200", "csrc", "rvq_encode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dist_topk_traffic.txt")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="image", choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--rows", type=int, default=None, help="smaller N with the same recipe (profiling)")
+    return p.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_label(spec):
+    return (f"{spec.name}: N={spec.N} D={spec.D} L={spec.L} K={spec.K}, "
+            f"{spec.f_dtype} features, {spec.cb_dtype} codebooks; {spec.description}")
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            time.sleep(0.15)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        busy = [v for v in sm if v > 0.5 * (mx or 0)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def gpu_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    return ids[local_rank] if local_rank < len(ids) else str(local_rank)
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def read_traffic(workload):
+    """ncu DRAM bytes per distance-GEMM launch for this workload, if captured from the current
+    kernel source (profiles/dist_topk_traffic.txt lines: workload bytes_per_launch source_sha)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    sha = file_sha(GEMM_KERNEL_SRC)
+    with open(TRAFFIC_FILE) as f:
+        for ln in f:
+            parts = ln.split()
+            if len(parts) >= 3 and not ln.startswith("#") and parts[0] == workload and parts[2] == sha:
+                return float(parts[1])
+    return None
+
+
+def cpu_baseline(g, seconds, rows_hint=None):
+    """The fp64 oracle, as it stands, on a bounded seeded row sample on this host's cores."""
+    import oracle
+    x, C = g["x"], g["codebooks"]
+    spec = g["spec"]
+    if x is None:  # detok: the CPU leg decodes
+        ids = g["planted"]
+        probe = workloads.sample_rows(len(ids), 256, seed=9)
+        t0 = time.perf_counter()
+        oracle.decode(ids[probe], C)
+        dt = max(time.perf_counter() - t0, 1e-6)
+        rows = min(len(ids), max(256, int(len(probe) * seconds / dt)))
+        sample = workloads.sample_rows(len(ids), rows, seed=10)
+        t0 = time.perf_counter()
+        oracle.decode(ids[sample], C)
+        dt = time.perf_counter() - t0
+    else:
+        cores = oracle.threads()
+        probe = workloads.sample_rows(len(x), cores, seed=8)
+        t0 = time.perf_counter()
+        oracle.encode(x, C, rows=probe)
+        dt = max(time.perf_counter() - t0, 1e-6)
+        rows = int(max(cores, min(len(x), len(probe) * seconds / dt)))
+        rows = max(1, min(len(x), rows if rows_hint is None else rows_hint))
+        sample = workloads.sample_rows(len(x), rows, seed=10)
+        t0 = time.perf_counter()
+        oracle.encode(x, C, rows=sample)
+        dt = time.perf_counter() - t0
+    value = len(sample) / dt / 1e6
+    return {"value": value, "unit": "Mtokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{len(sample)} of {spec.N} rows (seeded), full pipeline per row, "
+                      f"fp64 plain C + OpenMP over rows, {dt:.2f} s"}
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle timed on this host's cores, rank 0 only."""
+    if rank != 0:
+        return
+    g = workloads.generate(args.workload, n_override=args.rows)
+    spec = g["spec"]
+    per_step = max(0.5, min(args.cpu_seconds, 90.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    cb = None
+    for k in range(args.warmup + args.steps):
+        cb = cpu_baseline(g, per_step)
+        if k >= args.warmup:
+            vals.append(cb["value"])
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": spec.N / (value * 1e6) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_label(spec), "N": spec.N, "D": spec.D, "L": spec.L, "K": spec.K,
+                       "note": "fp64 oracle on host cores; each step a bounded seeded row sample; "
+                               "ms_per_step extrapolated to the full batch (rows are independent)"},
+            "cpu_baseline": dict(cb, value=value),
+            "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import multimodal_visual_tokenization_b200 as mvt
+    from multimodal_visual_tokenization_b200 import sharding
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+
+    g = workloads.generate(args.workload, batch=rank, n_override=args.rows)
+    spec = g["spec"]
+    N, D, L, K = spec.N, spec.D, spec.L, spec.K
+
+    def to_dev(a, dt):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.to(torch.bfloat16) if dt == "bf16" else t).to(dev)
+
+    cb = to_dev(g["codebooks"], spec.cb_dtype)
+    tok = mvt.Tokenizer(cb)
+    detok_only = g["x"] is None
+    if detok_only:
+        ids_in = torch.from_numpy(g["planted"]).to(dev)
+        x = tok.decode(ids_in)                       # fp32 features to re-encode
+        x_host_np = None
+    else:
+        x = to_dev(g["x"], spec.f_dtype)
+    f_code = mvt._dtype_code(x)
+    ids = torch.empty((N, L), dtype=torch.int32, device=dev)
+    res = torch.empty((N, D), dtype=torch.float32, device=dev)
+    rec = torch.empty((N, D), dtype=torch.float32, device=dev)
+    rec2 = torch.empty((N, D), dtype=torch.float32, device=dev)
+    fb = torch.zeros(L, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws, ws_bytes = tok.workspace(N)
+    off = torch.from_numpy(g["offsets"]).to(dev)
+    B = off.numel() - 1
+    stream = torch.cuda.current_stream(dev)
+
+    def check(code, what):
+        if code != 0:
+            raise mvt.RVQError(code, what)
+
+    def step(xin, dec_ids=None):
+        check(mvt.rvq_build_norms(cb, tok.cb_dtype, L, K, D, tok.norms, tok.level_stats, tok.operand, stream),
+              "rvq_build_norms")
+        check(mvt.rvq_encode(xin, f_code, N, D, cb, tok.cb_dtype, tok.operand, tok.norms, tok.level_stats, L, K,
+                             off, B, ids, res, rec, fb, ws, ws_bytes, status, stream), "rvq_encode")
+        check(mvt.rvq_decode(ids if dec_ids is None else dec_ids, N, L, cb, tok.cb_dtype, K, D, rec2, status,
+                             stream), "rvq_decode")
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize(dev)
+
+    # -------------------------------------------------- timed region, device-resident inputs
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_index(local_rank)) as clk:
+        mvt.rvq_profile_enable(True)
+        launches0 = mvt.rvq_launch_count()
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step(x)
+            ends[k].record(stream)
+        torch.cuda.synchronize(dev)
+        launches = mvt.rvq_launch_count() - launches0
+        code, gemm_n, gemm_ms = mvt.rvq_profile_read()
+        mvt.rvq_profile_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sharding.max_over_ranks(sum(step_ms), dev)
+    st = int(status.item())
+    if st != 0:
+        raise mvt.RVQError(st, "device status during the timed region")
+    ms_per_step = total_ms / args.steps
+    value = N * world / (ms_per_step / 1e3) / 1e6
+
+    # -------------------------------------------------- per-call breakdown (separate pass)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    br = {"norms": [], "encode": [], "decode": []}
+    for _ in range(min(args.steps, 20)):
+        flush.zero_()
+        ev[0].record(stream)
+        check(mvt.rvq_build_norms(cb, tok.cb_dtype, L, K, D, tok.norms, tok.level_stats, tok.operand, stream), "")
+        ev[1].record(stream)
+        check(mvt.rvq_encode(x, f_code, N, D, cb, tok.cb_dtype, tok.operand, tok.norms, tok.level_stats, L, K,
+                             off, B, ids, res, rec, fb, ws, ws_bytes, status, stream), "")
+        ev[2].record(stream)
+        check(mvt.rvq_decode(ids, N, L, cb, tok.cb_dtype, K, D, rec2, status, stream), "")
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        br["norms"].append(ev[0].elapsed_time(ev[1]))
+        br["encode"].append(ev[1].elapsed_time(ev[2]))
+        br["decode"].append(ev[2].elapsed_time(ev[3]))
+    breakdown = {k: statistics.median(v) for k, v in br.items()}
+    s_cb = 2 if spec.cb_dtype == "bf16" else 4
+    decode_bytes = N * L * 4 + L * K * D * s_cb + N * D * 4
+    decode_gbs = decode_bytes / (breakdown["decode"] / 1e3) / 1e9
+
+    # -------------------------------------------------- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        if detok_only:
+            h_in = torch.from_numpy(g["planted"]).pin_memory()
+            d_in = torch.empty_like(ids)
+        else:
+            h_in = (torch.from_numpy(g["x"]).to(torch.bfloat16) if spec.f_dtype == "bf16"
+                    else torch.from_numpy(g["x"])).pin_memory()
+            d_in = torch.empty_like(x)
+        h_ids = torch.empty((N, L), dtype=torch.int32).pin_memory()
+        h_rec = torch.empty((N, D), dtype=torch.float32).pin_memory()
+        e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for k in range(args.steps + 2):
+            flush.zero_()
+            kk = k - 2
+            if kk >= 0:
+                e_starts[kk].record(stream)
+            d_in.copy_(h_in, non_blocking=True)
+            if detok_only:
+                xin = tok.decode(d_in, out=x, check=False)
+                step(xin)
+            else:
+                step(d_in)
+            h_ids.copy_(ids, non_blocking=True)
+            h_rec.copy_(rec2, non_blocking=True)
+            if kk >= 0:
+                e_ends[kk].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sharding.max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), dev)
+        h2d = h_in.numel() * h_in.element_size()
+        d2h = h_ids.numel() * 4 + h_rec.numel() * 4
+        e2e = {"value": N * world / (e_ms / args.steps / 1e3) / 1e6, "unit": "Mtokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms / args.steps}
+
+    # -------------------------------------------------- roofline of the distance GEMM
+    long_step = ms_per_step > 20.0
+    peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
+    peak = float(peaks.get(peak_key, PEAKS_FALLBACK[peak_key]))
+    flops_per_launch = 2.0 * N * K * D  # one level: every (row, codeword) dot product
+    gemm_avg_ms = gemm_ms / max(1, gemm_n)
+    achieved = flops_per_launch / (gemm_avg_ms / 1e3) / 1e12
+    traffic = read_traffic(args.workload)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "dist_topk_kernel", "launch_ms": gemm_avg_ms,
+                "launches_timed": gemm_n, "flops_per_launch": flops_per_launch,
+                "peak_source": f"{peak_src} {peak_key}"}
+
+    # -------------------------------------------------- quick parity sample + CPU baseline
+    parity = None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rows = workloads.sample_rows(N, 6, seed=11)
+        xs = g["x"] if not detok_only else x.cpu().numpy()
+        want, _, _, _ = oracle.encode(xs, g["codebooks"], rows=rows)
+        got = ids.cpu().numpy()[rows]
+        parity = {"rows": int(len(rows)), "ids_equal_oracle": bool(np.array_equal(want, got))}
+        gg = dict(g)
+        if detok_only:
+            gg["x"] = xs
+        cpu = cpu_baseline(gg, args.cpu_seconds)
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_label(spec), "N": N, "D": D, "L": L, "K": K,
+                   "step": "rvq_build_norms + rvq_encode(ids, residual, recon) + rvq_decode",
+                   "l2": "flushed between timed steps (512 MiB memset, outside the step events)",
+                   "parallelism": f"replicas x{world}, rows independent, no data-path collective"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "breakdown_ms": breakdown,
+        "decode": {"GB_per_s": decode_gbs, "algorithmic_bytes": decode_bytes,
+                   "frac_hbm": decode_gbs / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))},
+        "fallbacks_per_level": fb.cpu().tolist(),
+        "parity_sample": parity,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
