@@ -71,7 +71,8 @@ typedef enum {
  * rvq_build_norms -- one-off preparation of a fixed codebook set ("Offline Visual
  * Preprocessing": the tokenizer is fixed, so this runs once per codebook set).
  *   codebooks    [L, K, D] in cb_dtype
- *   norms        [L, K] fp32 out: ||C_l[k]||^2, accumulated in fp64, rounded to nearest
+ *   norms        [L, K] fp32 out: ||C_l[k]||^2 (fp32 lane sums of <= ceil(D/32) squares, combined
+ *                in fp64, rounded to nearest: relative error <= (D/32+2) 2^-24)
  *   level_stats  [L, RVQ_LEVEL_STATS] fp32 out (see above)
  *   cb_operand   [L, K, D] bf16 out: round-to-nearest-even copy used as the tensor-core
  *                operand.  Required when cb_dtype == RVQ_F32; ignored (may be NULL) for

@@ -38,9 +38,11 @@ class RVQError(RuntimeError):
         self.code = code
 
 
-def load(path: str = LIB_PATH):
-    """Load librvq.so (built by `python -m multimodal_visual_tokenization_b200._build`)."""
+def load(path: str | None = None):
+    """Load librvq.so (built by `python -m multimodal_visual_tokenization_b200._build`).
+    RVQ_LIBRARY names another build of the same library (e.g. a tuning variant)."""
     global _lib
+    path = path or os.environ.get("RVQ_LIBRARY") or LIB_PATH
     with _lock:
         if _lib is not None:
             return _lib

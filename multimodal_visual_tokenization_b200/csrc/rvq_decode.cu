@@ -2,10 +2,11 @@
 // Figure 1: discrete token sequences are turned back into features for the visual
 // de-tokenizer).  HBM-bound: ids are read, recon is written once, codebook rows are gathered.
 //
-// Schedule: the feature axis is cut into 128-column slices and the grid runs slice-major
-// (blockIdx.y = slice), so while one slice is being produced only L*K*128 codebook elements
-// are live; they stay resident in L2 and DRAM sees each codebook byte about once.  recon is
-// written with streaming stores so it does not evict those codebook lines.
+// Schedule: the feature axis is cut into slices of 32 x (16-byte load) columns and the grid runs
+// slice-major (blockIdx.y = slice), so while one slice is being produced only L*K*slice codebook
+// elements are live; they stay resident in L2 and DRAM sees each codebook byte about once.
+// recon is written with streaming stores so it does not evict those codebook lines.  Gathers of
+// eight levels are in flight at once per warp to cover L2 latency.
 #include <cuda_bf16.h>
 
 #include "rvq_device.cuh"
@@ -13,87 +14,135 @@
 
 namespace rvq {
 
-constexpr int kDecodeRowsPerWarp = 4;
 constexpr int kDecodeWarps = 8;
-constexpr int kDecodeSlice = 128;  // columns per slice: 32 lanes x 4
+constexpr int kDecodeLevelGroup = 8;  // gathers issued together before they are summed
 
-template <bool CB_BF16>
-__device__ __forceinline__ float4 load4(const void *cb, int64_t off) {
-  if constexpr (CB_BF16) {
-    uint2 raw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(cb) + off));
-    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
-    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
-    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-    return make_float4(fa.x, fa.y, fb.x, fb.y);
-  } else {
-    return __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(cb) + off));
+// VEC consecutive elements of one codeword row, widened to fp32.
+template <bool CB_BF16, int VEC>
+struct Gather;
+
+template <>
+struct Gather<true, 8> {  // 16-byte load of 8 bf16
+  uint4 raw;
+  __device__ __forceinline__ void load(const void *cb, int64_t off) {
+    raw = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(cb) + off));
   }
-}
+  __device__ __forceinline__ void zero() { raw = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void add_to(float *acc) const {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
+      acc[2 * k] += f.x;
+      acc[2 * k + 1] += f.y;
+    }
+  }
+};
 
-template <bool CB_BF16>
+template <>
+struct Gather<true, 4> {  // 8-byte load of 4 bf16 (D not a multiple of 8)
+  uint2 raw;
+  __device__ __forceinline__ void load(const void *cb, int64_t off) {
+    raw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(cb) + off));
+  }
+  __device__ __forceinline__ void zero() { raw = make_uint2(0, 0); }
+  __device__ __forceinline__ void add_to(float *acc) const {
+    const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
+      acc[2 * k] += f.x;
+      acc[2 * k + 1] += f.y;
+    }
+  }
+};
+
+template <>
+struct Gather<false, 4> {  // 16-byte load of 4 fp32
+  float4 raw;
+  __device__ __forceinline__ void load(const void *cb, int64_t off) {
+    raw = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(cb) + off));
+  }
+  __device__ __forceinline__ void zero() { raw = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void add_to(float *acc) const {
+    acc[0] += raw.x;
+    acc[1] += raw.y;
+    acc[2] += raw.z;
+    acc[3] += raw.w;
+  }
+};
+
+// One warp per row and slice of 32*VEC columns; lane = VEC consecutive columns.  The gathers of
+// eight levels are issued back to back with no branch between them (an out-of-range id or a
+// lane past D reads a clamped, valid address and is masked afterwards), then summed in
+// ascending level order.
+template <bool CB_BF16, int VEC>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t *__restrict__ ids, int64_t N,
                                                                   int L, const void *__restrict__ cb, int K,
                                                                   int D, float *__restrict__ recon,
                                                                   int32_t *status) {
-  constexpr int R = kDecodeRowsPerWarp;
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int col = blockIdx.y * kDecodeSlice + lane * 4;
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * kDecodeWarps + (threadIdx.x >> 5);
+  if (n >= N) return;  // whole warp
+  const int col = blockIdx.y * (32 * VEC) + lane * VEC;
   const bool active = col < D;
-  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * kDecodeWarps + warp) * R;
-
-  // lane j holds the ids of levels j and 32+j for each of the warp's rows
-  int id_lo[R], id_hi[R];
+  const int colc = active ? col : 0;
+  const int32_t *row_ids = ids + n * L;
+  const int id_lo = lane < L ? __ldg(row_ids + lane) : 0;
+  const int id_hi = lane + 32 < L ? __ldg(row_ids + 32 + lane) : 0;
+  float acc[VEC];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int64_t n = row0 + r;
-    id_lo[r] = (n < N && lane < L) ? __ldg(ids + n * L + lane) : 0;
-    id_hi[r] = (n < N && lane + 32 < L) ? __ldg(ids + n * L + 32 + lane) : 0;
-  }
-  float4 acc[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
   bool bad = false;
-#pragma unroll 2
-  for (int l = 0; l < L; ++l) {
-    const int64_t lbase = static_cast<int64_t>(l) * K;
+  for (int l0 = 0; l0 < L; l0 += kDecodeLevelGroup) {
+    Gather<CB_BF16, VEC> g[kDecodeLevelGroup];
+    bool use[kDecodeLevelGroup];
+    const int src = l0 < 32 ? id_lo : id_hi;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int id = l < 32 ? __shfl_sync(0xffffffffu, id_lo[r], l) : __shfl_sync(0xffffffffu, id_hi[r], l - 32);
-      const bool row_ok = row0 + r < N;
-      const bool in_range = static_cast<unsigned>(id) < static_cast<unsigned>(K);
-      bad |= row_ok && !in_range;
-      if (row_ok && in_range && active) {
-        float4 c = load4<CB_BF16>(cb, (lbase + id) * D + col);
-        acc[r].x += c.x;
-        acc[r].y += c.y;
-        acc[r].z += c.z;
-        acc[r].w += c.w;
-      }
+    for (int j = 0; j < kDecodeLevelGroup; ++j) {
+      const int l = l0 + j;
+      const int id = __shfl_sync(0xffffffffu, src, l & 31);
+      const bool lv = l < L;
+      const bool ok = lv && static_cast<unsigned>(id) < static_cast<unsigned>(K);
+      bad |= lv && !ok;
+      use[j] = ok;
+      const int lc = lv ? l : L - 1;
+      g[j].load(cb, (static_cast<int64_t>(lc) * K + (ok ? id : 0)) * D + colc);
     }
+#pragma unroll
+    for (int j = 0; j < kDecodeLevelGroup; ++j)
+      if (use[j]) g[j].add_to(acc);
   }
   if (active) {
+    float4 *dst = reinterpret_cast<float4 *>(recon + n * D + col);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int64_t n = row0 + r;
-      if (n < N) __stcs(reinterpret_cast<float4 *>(recon + n * D + col), acc[r]);
-    }
+    for (int k = 0; k < VEC; k += 4) __stcs(dst + k / 4, make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]));
   }
   if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
+}
+
+template <bool CB_BF16, int VEC>
+void launch_decode_t(const int32_t *ids, int64_t N, int L, const void *cb, int K, int D, float *recon,
+                     int32_t *status, cudaStream_t s, dim3 grid) {
+  decode_kernel<CB_BF16, VEC><<<grid, kDecodeWarps * 32, 0, s>>>(ids, N, L, cb, K, D, recon, status);
 }
 
 int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_dtype, int K, int D, float *recon,
                   int32_t *status, cudaStream_t s) {
   if (N == 0) return RVQ_OK;
-  const int64_t rows_per_block = static_cast<int64_t>(kDecodeWarps) * kDecodeRowsPerWarp;
-  const int64_t gx = (N + rows_per_block - 1) / rows_per_block;
-  const int gy = (D + kDecodeSlice - 1) / kDecodeSlice;
+  const int vec = (cb_dtype == RVQ_BF16 && D % 8 == 0) ? 8 : 4;
+  const int64_t gx = (N + kDecodeWarps - 1) / kDecodeWarps;
+  const int gy = (D + 32 * vec - 1) / (32 * vec);
   if (gx > 0x7FFFFFFFLL || gy > 65535) return RVQ_ERR_UNSUPPORTED;
-  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
-  if (cb_dtype == RVQ_BF16)
-    decode_kernel<true><<<grid, kDecodeWarps * 32, 0, s>>>(ids, N, L, cb, K, D, recon, status);
-  else
-    decode_kernel<false><<<grid, kDecodeWarps * 32, 0, s>>>(ids, N, L, cb, K, D, recon, status);
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  if (cb_dtype == RVQ_BF16) {
+    if (vec == 8)
+      launch_decode_t<true, 8>(ids, N, L, cb, K, D, recon, status, s, grid);
+    else
+      launch_decode_t<true, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
+  } else {
+    launch_decode_t<false, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
+  }
   note_launch();
   return check_launch();
 }

@@ -29,7 +29,7 @@
 // Error bound used by the certificate, per row and level (r fp32 residual, r~ = bf16(r),
 // c stored codeword, c~ = bf16(c), n = fl32(||c||^2), s~ = tensor-core r~.c~ with fp32
 // accumulation, gamma = (D+16) 2^-22):
-//   | (||r-c||^2 - ||r||^2) - d~ | <= 2^-22 Nmax + 2 (||r-r~|| Cmax + ||r~|| dCmax)
+//   | (||r-c||^2 - ||r||^2) - d~ | <= (D/32+2) 2^-24 Nmax + 2 (||r-r~|| Cmax + ||r~|| dCmax)
 //                                     + 2 gamma ||r~|| C~max + 2^-23 (Nmax + 2 ||r~|| C~max)
 // where Cmax, dCmax, C~max, Nmax are the per-level maxima of ||c||, ||c-c~||, ||c~||, n from
 // rvq_build_norms (Cauchy-Schwarz on the two rounding error vectors, worst-case summation error
@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "rvq_device.cuh"
@@ -57,17 +58,31 @@ constexpr int BK = 64;        // bf16 elements per k-block = one 128-byte swizzl
 constexpr int UK = 16;        // K of one kind::f16 UMMA
 constexpr int NSTAGE = 4;
 constexpr int TOPK = 8;
-constexpr int MAX_CAND = 64;  // candidates the rescore warp can merge (2 per lane)
+constexpr int MAX_SLOTS = 8;  // partial lists per row tile (bounds the rescore merge)
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int GEMM_THREADS = 192;  // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
-constexpr int SMEM_BARRIER_OFF = NSTAGE * STAGE_BYTES;
-constexpr int GEMM_SMEM = SMEM_BARRIER_OFF + 256 + 1024;  // + barriers + alignment slack
 
 __device__ __forceinline__ float inf_f() { return __int_as_float(0x7f800000); }
 __device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
+
+// Thread organisation of the distance-GEMM block: EPI epilogue warps (EPI/4 column groups x 4
+// TMEM lane quadrants), then one TMA producer warp and one MMA-issuer warp.
+template <int EPI>
+struct GemmCfg {
+  static constexpr int GROUPS = EPI / 4;
+  static constexpr int COLS = BN / GROUPS;  // columns of a tile one epilogue thread scans
+  static constexpr int CHUNKS = COLS / 32;
+  static constexpr int EPI_THREADS = EPI * 32;
+  static constexpr int THREADS = EPI_THREADS + 64;
+  static constexpr int PRODUCER = EPI;
+  static constexpr int ISSUER = EPI + 1;
+  static constexpr int NORM_OFF = NSTAGE * STAGE_BYTES;                  // 2 x 256 fp32 norms
+  static constexpr int MERGE_OFF = NORM_OFF + 2 * BN * 4;                // (GROUPS-1) x 128 x 8 x 8 B
+  static constexpr int BAR_OFF = MERGE_OFF + (GROUPS - 1) * BM * TOPK * 8;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;                      // + barriers + alignment slack
+};
 
 struct GemmArgs {
   const float *norms;  // [K] of this level
@@ -78,6 +93,7 @@ struct GemmArgs {
   int Tc;     // codeword tiles
   int G;      // CTAs
   int maxs;   // partial-list slots per row tile
+  int bulk_norms;  // norms staged by bulk copy (K % 4 == 0)
   float2 *cand;
   int32_t *status;
 };
@@ -87,41 +103,44 @@ __host__ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t U, int G)
   return static_cast<int>(((u + 1) * static_cast<int64_t>(G) - 1) / U);
 }
 
+// Insert (x, ix) into the ascending list bd/bi, dropping the largest entry.  Entries equal to x
+// stay ahead of it (first seen wins).  Written as independent compares + selects so the update
+// has a short dependency chain.
 __device__ __forceinline__ void topk_insert(float (&bd)[TOPK], int (&bi)[TOPK], float x, int ix) {
+  bool c[TOPK];
 #pragma unroll
-  for (int t = 0; t < TOPK; ++t) {
-    const bool sw = x < bd[t];
-    const float tb = bd[t];
-    const int ti = bi[t];
-    bd[t] = sw ? x : tb;
-    bi[t] = sw ? ix : ti;
-    x = sw ? tb : x;
-    ix = sw ? ti : ix;
+  for (int t = 0; t < TOPK; ++t) c[t] = bd[t] <= x;
+#pragma unroll
+  for (int t = TOPK - 1; t >= 1; --t) {
+    const float nb = c[t] ? bd[t] : (c[t - 1] ? x : bd[t - 1]);
+    const int ni = c[t] ? bi[t] : (c[t - 1] ? ix : bi[t - 1]);
+    bd[t] = nb;
+    bi[t] = ni;
+  }
+  if (!c[0]) {
+    bd[0] = x;
+    bi[0] = ix;
   }
 }
 
-// Write one row's partial top-8 list for row tile rt into this CTA's slot.
-__device__ __forceinline__ void flush_topk(const GemmArgs &a, int64_t rt, int row_in_tile, const float (&bd)[TOPK],
-                                           const int (&bi)[TOPK]) {
-  const int64_t n = rt * BM + row_in_tile;
-  if (n < a.N) {
-    const int slot = static_cast<int>(blockIdx.x) - cta_of_unit(rt * a.Tc, a.U, a.G);
-    float2 *out = a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK;
-#pragma unroll
-    for (int t = 0; t < TOPK; ++t) out[t] = make_float2(bd[t], __int_as_float(bi[t]));
-  }
-}
-
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <int EPI>
+__global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     dist_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs a) {
+  using C = GemmCfg<EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SMEM_BARRIER_OFF);
+  float *nslot = reinterpret_cast<float *>(smem + C::NORM_OFF);
+  float2 *mbuf = reinterpret_cast<float2 *>(smem + C::MERGE_OFF);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint64_t *empty = full + NSTAGE;
   uint64_t *tfull = empty + NSTAGE;
   uint64_t *tempty = tfull + 2;
-  uint64_t *mma_done = tempty + 2;
+  uint64_t *nfull = tempty + 2;
+  uint64_t *nempty = nfull + 2;
+  uint64_t *mready = nempty + 2;
+  uint64_t *mdone = mready + 1;
+  uint64_t *mma_done = mdone + 1;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
   volatile int *never = abort_flag + 1;
@@ -139,14 +158,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], BM);
+      mbar_init(&tempty[b], C::EPI_THREADS);
+      mbar_init(&nfull[b], 1);
+      mbar_init(&nempty[b], C::EPI_THREADS);
     }
+    mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
+    mbar_init(mdone, 128);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     *never = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == C::ISSUER) {
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
@@ -155,7 +178,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == C::PRODUCER) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
@@ -164,9 +187,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t ph = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int64_t u = u0; u < u1 && ok; ++u) {
+      int64_t i = 0;
+      for (int64_t u = u0; u < u1 && ok; ++u, ++i) {
         const int64_t rt = u / a.Tc;
         const int ct = static_cast<int>(u - rt * a.Tc);
+        if (a.bulk_norms) {
+          const int slot = static_cast<int>(i & 1);
+          if (!mbar_wait(&nempty[slot], static_cast<uint32_t>((i >> 1) & 1) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int nvalid = min(BN, a.K - ct * BN);  // a multiple of 4 when bulk_norms
+          mbar_arrive_expect_tx(&nfull[slot], static_cast<uint32_t>(nvalid * 4));
+          bulk_load(nslot + slot * BN, a.norms + static_cast<int64_t>(ct) * BN, static_cast<uint32_t>(nvalid * 4),
+                    &nfull[slot]);
+        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
@@ -197,9 +232,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           mbar_wait(&full[back], p, never);
         }
+        if (a.bulk_norms && i > 0) {
+          for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
+            mbar_wait(&nfull[j & 1], static_cast<uint32_t>((j >> 1) & 1), never);
+        }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == C::ISSUER) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
@@ -247,9 +286,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue: running top-8
-    const int row_in_tile = warp * 32 + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-    const bool vec_norms = (a.K & 3) == 0;
+    const int quad = warp & 3;
+    const int grp = warp >> 2;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     float bd[TOPK];
     int bi[TOPK];
 #pragma unroll
@@ -259,12 +299,53 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     int64_t cur_rt = -1;
     int64_t i = 0;
+    uint32_t nflush = 0;
     bool ok = true;
+
+    // Merge the column groups' lists of row tile rt (group 0 gathers) and write it to this CTA's slot.
+    auto flush = [&](int64_t rt) -> bool {
+      if constexpr (C::GROUPS > 1) {
+        float2 *mine = mbuf + (static_cast<int64_t>(grp - 1) * BM + row_in_tile) * TOPK;
+        if (grp > 0) {
+          if (nflush > 0 && !mbar_wait(mdone, (nflush - 1) & 1u, abort_flag)) return false;
+#pragma unroll
+          for (int t = 0; t < TOPK; ++t) mine[t] = make_float2(bd[t], __int_as_float(bi[t]));
+          mbar_arrive(mready);
+        } else {
+          if (!mbar_wait(mready, nflush & 1u, abort_flag)) return false;
+          for (int gg = 1; gg < C::GROUPS; ++gg) {
+            const float2 *other = mbuf + (static_cast<int64_t>(gg - 1) * BM + row_in_tile) * TOPK;
+#pragma unroll
+            for (int t = 0; t < TOPK; ++t) {
+              const float2 e = other[t];
+              if (e.x < bd[TOPK - 1]) topk_insert(bd, bi, e.x, __float_as_int(e.y));
+            }
+          }
+          mbar_arrive(mdone);
+        }
+      }
+      ++nflush;
+      if (grp == 0) {
+        const int64_t n = rt * BM + row_in_tile;
+        if (n < a.N) {
+          const int slot = static_cast<int>(blockIdx.x) - cta_of_unit(rt * a.Tc, a.U, a.G);
+          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK);
+#pragma unroll
+          for (int t = 0; t < TOPK; t += 2)
+            out[t / 2] = make_float4(bd[t], __int_as_float(bi[t]), bd[t + 1], __int_as_float(bi[t + 1]));
+        }
+      }
+      return true;
+    };
+
     for (int64_t u = u0; u < u1; ++u, ++i) {
       const int64_t rt = u / a.Tc;
       const int ct = static_cast<int>(u - rt * a.Tc);
       if (rt != cur_rt) {
-        if (cur_rt >= 0) flush_topk(a, cur_rt, row_in_tile, bd, bi);
+        if (cur_rt >= 0 && !flush(cur_rt)) {
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int t = 0; t < TOPK; ++t) {
           bd[t] = inf_f();
@@ -274,7 +355,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       const int buf = static_cast<int>(i & 1);
       const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
-      const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
+      bool got = mbar_wait(&tfull[buf], tph, abort_flag);
+      if (got && a.bulk_norms) got = mbar_wait(&nfull[buf], tph, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
@@ -284,21 +366,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int col0 = ct * BN;
       const int nvalid = min(BN, a.K - col0);
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = 0; ch < C::CHUNKS; ++ch) {
+        const int ct0 = grp * C::COLS + ch * 32;  // first column of the chunk within the tile
         uint32_t v[32];
-        tmem_ld_32x32(lane_base + static_cast<uint32_t>(buf * BN + ch * 32), v);
+        tmem_ld_32x32(lane_base + static_cast<uint32_t>(buf * BN + ct0), v);
         tmem_ld_wait();
-        if (ch == BN / 32 - 1) {
+        if (ch == C::CHUNKS - 1) {
           tc_fence_before();
           mbar_arrive(&tempty[buf]);
         }
-        const int c0 = col0 + ch * 32;
+        const int c0 = col0 + ct0;
         float d[32];
-        if (ch * 32 + 32 <= nvalid && vec_norms) {
-          const float4 *np = reinterpret_cast<const float4 *>(a.norms + c0);
+        if (a.bulk_norms && ct0 + 32 <= nvalid) {
+          const float4 *np = reinterpret_cast<const float4 *>(nslot + buf * BN + ct0);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 nn = __ldg(np + j);
+            const float4 nn = np[j];
             d[4 * j + 0] = fmaf(-2.f, __uint_as_float(v[4 * j + 0]), nn.x);
             d[4 * j + 1] = fmaf(-2.f, __uint_as_float(v[4 * j + 1]), nn.y);
             d[4 * j + 2] = fmaf(-2.f, __uint_as_float(v[4 * j + 2]), nn.z);
@@ -307,31 +390,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            d[j] = (ch * 32 + j < nvalid) ? fmaf(-2.f, __uint_as_float(v[j]), __ldg(a.norms + c0 + j)) : inf_f();
+            d[j] = (ct0 + j < nvalid) ? fmaf(-2.f, __uint_as_float(v[j]), __ldg(a.norms + c0 + j)) : inf_f();
         }
-        float m = d[0];
+        // chunk minimum as a tree (short dependency chain)
+        float m16[16];
 #pragma unroll
-        for (int j = 1; j < 32; ++j) m = fminf(m, d[j]);
-        if (__any_sync(0xffffffffu, m < bd[TOPK - 1])) {
+        for (int j = 0; j < 16; ++j) m16[j] = fminf(d[j], d[j + 16]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int j = 0; j < w; ++j) m16[j] = fminf(m16[j], m16[j + w]);
+        if (__any_sync(0xffffffffu, m16[0] < bd[TOPK - 1])) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (__any_sync(0xffffffffu, d[j] < bd[TOPK - 1])) topk_insert(bd, bi, d[j], c0 + j);
           }
         }
       }
+      if (a.bulk_norms) mbar_arrive(&nempty[buf]);
     }
+    if (ok && cur_rt >= 0 && !flush(cur_rt)) ok = false;
     if (!ok) {
       *abort_flag = 1;
       set_status(a.status, RVQ_ERR_TIMEOUT);
-    } else if (cur_rt >= 0) {
-      flush_topk(a, cur_rt, row_in_tile, bd, bi);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == C::ISSUER) {
     __syncwarp();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -444,8 +532,10 @@ struct RowArgs {
 __device__ __forceinline__ float error_bound(const float *st, float2 rs, int D) {
   const float cmax = st[0], dcmax = st[1], cqmax = st[2], nmax = st[3];
   const float gamma = static_cast<float>(D + 16) * 2.384185791015625e-07f;  // 2^-22
-  const float e = 2.384185791015625e-07f * nmax + 2.f * (rs.x * cmax + rs.y * dcmax) +
-                  2.f * gamma * rs.y * cqmax + 1.1920928955078125e-07f * (nmax + 2.f * rs.y * cqmax);
+  // norms: fp32 lane sums of ceil(D/32) squares combined in fp64, then rounded to fp32
+  const float norm_err = static_cast<float>(D / 32 + 2) * 5.9604644775390625e-08f;  // (D/32+2) 2^-24
+  const float e = norm_err * nmax + 2.f * (rs.x * cmax + rs.y * dcmax) + 2.f * gamma * rs.y * cqmax +
+                  1.1920928955078125e-07f * (nmax + 2.f * rs.y * cqmax);
   return 1.01f * e;
 }
 
@@ -641,7 +731,7 @@ inline Plan make_plan(int64_t N, int K, int sms) {
   p.U = p.RT * p.Tc;
   // every CTA covers at least f = floor(U/G) units, so a row tile (Tc consecutive units) meets
   // at most 1 + ceil((Tc-1)/f) CTAs; keep that within the rescore warp's candidate capacity
-  const int64_t slots_cap = MAX_CAND / TOPK;
+  const int64_t slots_cap = MAX_SLOTS;
   const int64_t need_f = std::max<int64_t>(1, (p.Tc - 1 + slots_cap - 2) / (slots_cap - 1));
   int64_t G = std::min<int64_t>(sms, p.U);
   G = std::min<int64_t>(G, std::max<int64_t>(1, p.U / need_f));
@@ -706,6 +796,44 @@ inline bool make_map(CUtensorMap *m, const void *base, int64_t rows, int D, int 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+template <int EPI>
+inline bool set_gemm_attr() {
+  return cudaFuncSetAttribute(dist_topk_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<EPI>::SMEM) == cudaSuccess;
+}
+
+// Epilogue warps of the distance GEMM.  A short feature width gives little MMA time per tile to
+// hide the epilogue behind, so more warps share it (measured: 16 warps win at D <= 256, 8 above).
+// RVQ_EPI_WARPS=4|8|16 overrides the choice (tuning knob).
+inline int epilogue_warps(int D) {
+  static int forced = [] {
+    const char *e = getenv("RVQ_EPI_WARPS");
+    const int v = e ? atoi(e) : 0;
+    return (v == 4 || v == 8 || v == 16) ? v : 0;
+  }();
+  if (forced) return forced;
+  return D <= 256 ? 16 : 8;
+}
+
+inline bool gemm_attrs_ready(int epi) {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] { ok = set_gemm_attr<4>() && set_gemm_attr<8>() && set_gemm_attr<16>(); });
+  (void)epi;
+  return ok;
+}
+
+inline void launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                        const GemmArgs &ga) {
+  if (epi == 4)
+    dist_topk_kernel<4><<<grid, GemmCfg<4>::THREADS, GemmCfg<4>::SMEM, s>>>(tmA, tmB, ga);
+  else if (epi == 16)
+    dist_topk_kernel<16><<<grid, GemmCfg<16>::THREADS, GemmCfg<16>::SMEM, s>>>(tmA, tmB, ga);
+  else
+    dist_topk_kernel<8><<<grid, GemmCfg<8>::THREADS, GemmCfg<8>::SMEM, s>>>(tmA, tmB, ga);
+}
+
 }  // namespace enc
 }  // namespace rvq
 
@@ -760,13 +888,8 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   CUtensorMap tmA;
   if (!make_map(&tmA, Rt, N, D, BM)) return RVQ_ERR_CUDA;
 
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(dist_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM) !=
-        cudaSuccess)
-      return RVQ_ERR_CUDA;
-    attr_done = true;
-  }
+  const int epi = epilogue_warps(D);
+  if (!gemm_attrs_ready(epi)) return RVQ_ERR_CUDA;
 
   {
     const int64_t threads = N * 32;
@@ -800,7 +923,8 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ga.cand = cand;
     ga.status = status;
     profile_begin(s);
-    dist_topk_kernel<<<p.G, GEMM_THREADS, GEMM_SMEM, s>>>(tmA, tmB, ga);
+    ga.bulk_norms = (K % 4) == 0 ? 1 : 0;
+    launch_gemm(epi, p.G, s, tmA, tmB, ga);
     profile_end(s);
     note_launch();
     if ((st = check_launch()) != RVQ_OK) return st;

@@ -14,63 +14,105 @@ __device__ __forceinline__ void atomic_max_nonneg(float *addr, float v) {
   atomicMax(reinterpret_cast<unsigned int *>(addr), __float_as_uint(v));
 }
 
-// One warp per codeword.  Lanes stride over D in chunks of 4 elements.
+// One warp per codeword, eight codewords per block.  Each lane accumulates its strided share
+// of the row in fp32 (at most D/32 terms), lane sums are combined in fp64; the per-level maxima
+// are reduced in the block first so only one atomic per block and statistic reaches L2.
 template <bool CB_BF16>
 __global__ void __launch_bounds__(256) norms_kernel(const void *__restrict__ cb, int L, int K, int D,
                                                     float *__restrict__ norms, float *__restrict__ stats,
                                                     __nv_bfloat16 *__restrict__ cb_op) {
+  __shared__ float wmax[8][RVQ_LEVEL_STATS];
+  __shared__ int wlev[8];
   const int lane = threadIdx.x & 31;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int warp = threadIdx.x >> 5;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + warp;
   const int64_t total = static_cast<int64_t>(L) * K;
-  if (w >= total) return;
-  const int l = static_cast<int>(w / K);
-  double s_c = 0.0, s_q = 0.0, s_e = 0.0;  // ||c||^2, ||bf16(c)||^2, ||c - bf16(c)||^2
-  if constexpr (CB_BF16) {
-    const __nv_bfloat16 *row = static_cast<const __nv_bfloat16 *>(cb) + w * D;
-    for (int i = lane * 4; i < D; i += 128) {
-      uint2 raw = *reinterpret_cast<const uint2 *>(row + i);
-      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+  const bool live = w < total;
+  float s_c = 0.f, s_q = 0.f, s_e = 0.f;  // lane shares of ||c||^2, ||bf16(c)||^2, ||c - bf16(c)||^2
+  if (live) {
+    if constexpr (CB_BF16) {
+      const __nv_bfloat16 *row = static_cast<const __nv_bfloat16 *>(cb) + w * D;
+      for (int i0 = lane * 8; i0 < D; i0 += 1024) {
+        uint4 raw[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float2 f = __bfloat1622float2(h[j]);
-        s_c += static_cast<double>(f.x) * f.x + static_cast<double>(f.y) * f.y;
+        for (int u = 0; u < 4; ++u) {  // four 16-byte loads in flight per lane
+          const int i = i0 + u * 256;
+          raw[u] = (i + 8 <= D) ? __ldg(reinterpret_cast<const uint4 *>(row + i)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t wd[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wd[k]));
+            s_c = fmaf(f.x, f.x, s_c);
+            s_c = fmaf(f.y, f.y, s_c);
+          }
+        }
+      }
+      s_q = s_c;
+    } else {
+      const float *row = static_cast<const float *>(cb) + w * D;
+      __nv_bfloat16 *orow = cb_op + w * D;
+      for (int i0 = lane * 4; i0 < D; i0 += 512) {
+        float4 f[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // four 16-byte loads in flight per lane
+          const int i = i0 + u * 128;
+          f[u] = i < D ? __ldg(reinterpret_cast<const float4 *>(row + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * 128;
+          if (i >= D) break;
+          const __nv_bfloat162 a = __floats2bfloat162_rn(f[u].x, f[u].y);
+          const __nv_bfloat162 b = __floats2bfloat162_rn(f[u].z, f[u].w);
+          const float2 qa = __bfloat1622float2(a), qb = __bfloat1622float2(b);
+          const float v[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+          const float q[4] = {qa.x, qa.y, qb.x, qb.y};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            s_c = fmaf(v[k], v[k], s_c);
+            s_q = fmaf(q[k], q[k], s_q);
+            const float e = v[k] - q[k];  // exact: the bf16 rounding error of an fp32 value
+            s_e = fmaf(e, e, s_e);
+          }
+          uint2 packed;
+          packed.x = *reinterpret_cast<const uint32_t *>(&a);
+          packed.y = *reinterpret_cast<const uint32_t *>(&b);
+          *reinterpret_cast<uint2 *>(orow + i) = packed;
+        }
       }
     }
-    s_q = s_c;
-  } else {
-    const float *row = static_cast<const float *>(cb) + w * D;
-    __nv_bfloat16 *orow = cb_op + w * D;
-    for (int i = lane * 4; i < D; i += 128) {
-      float4 f = *reinterpret_cast<const float4 *>(row + i);
-      __nv_bfloat162 a = __floats2bfloat162_rn(f.x, f.y);
-      __nv_bfloat162 b = __floats2bfloat162_rn(f.z, f.w);
-      float2 qa = __bfloat1622float2(a), qb = __bfloat1622float2(b);
-      s_c += static_cast<double>(f.x) * f.x + static_cast<double>(f.y) * f.y + static_cast<double>(f.z) * f.z +
-             static_cast<double>(f.w) * f.w;
-      s_q += static_cast<double>(qa.x) * qa.x + static_cast<double>(qa.y) * qa.y +
-             static_cast<double>(qb.x) * qb.x + static_cast<double>(qb.y) * qb.y;
-      double e0 = static_cast<double>(f.x) - qa.x, e1 = static_cast<double>(f.y) - qa.y;
-      double e2 = static_cast<double>(f.z) - qb.x, e3 = static_cast<double>(f.w) - qb.y;
-      s_e += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
-      uint2 packed;
-      packed.x = *reinterpret_cast<uint32_t *>(&a);
-      packed.y = *reinterpret_cast<uint32_t *>(&b);
-      *reinterpret_cast<uint2 *>(orow + i) = packed;
-    }
   }
+  double dc = s_c, dq = s_q, de = s_e;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    s_c += __shfl_xor_sync(0xffffffffu, s_c, o);
-    s_q += __shfl_xor_sync(0xffffffffu, s_q, o);
-    s_e += __shfl_xor_sync(0xffffffffu, s_e, o);
+    dc += __shfl_xor_sync(0xffffffffu, dc, o);
+    dq += __shfl_xor_sync(0xffffffffu, dq, o);
+    de += __shfl_xor_sync(0xffffffffu, de, o);
   }
   if (lane == 0) {
-    norms[w] = __double2float_rn(s_c);
-    float *st = stats + static_cast<int64_t>(l) * RVQ_LEVEL_STATS;
-    atomic_max_nonneg(st + 0, __double2float_ru(sqrt(s_c)));
-    atomic_max_nonneg(st + 1, __double2float_ru(sqrt(s_e)));
-    atomic_max_nonneg(st + 2, __double2float_ru(sqrt(s_q)));
-    atomic_max_nonneg(st + 3, __double2float_ru(s_c));
+    wlev[warp] = live ? static_cast<int>(w / K) : -1;
+    if (live) {
+      norms[w] = __double2float_rn(dc);
+      wmax[warp][0] = __double2float_ru(sqrt(dc));
+      wmax[warp][1] = __double2float_ru(sqrt(de));
+      wmax[warp][2] = __double2float_ru(sqrt(dq));
+      wmax[warp][3] = __double2float_ru(dc);
+    }
+  }
+  __syncthreads();
+  // thread (warp j, stat k) publishes warp j's maximum unless an earlier warp of the block is
+  // on the same level, in which case that warp's thread folds it in
+  if (threadIdx.x < 8 * RVQ_LEVEL_STATS) {
+    const int j = threadIdx.x / RVQ_LEVEL_STATS, k = threadIdx.x % RVQ_LEVEL_STATS;
+    const int lev = wlev[j];
+    if (lev >= 0 && (j == 0 || wlev[j - 1] != lev)) {
+      float m = wmax[j][k];
+      for (int jj = j + 1; jj < 8 && wlev[jj] == lev; ++jj) m = fmaxf(m, wmax[jj][k]);
+      atomic_max_nonneg(stats + static_cast<int64_t>(lev) * RVQ_LEVEL_STATS + k, m);
+    }
   }
 }
 

@@ -217,7 +217,8 @@ def test_norms_and_stats():
     torch.cuda.synchronize()
     n = tok.norms.cpu().numpy().astype(np.float64)
     want = (C.astype(np.float64) ** 2).sum(-1)
-    assert np.allclose(n, want, rtol=2 ** -23, atol=0)
+    D = C.shape[2]
+    assert np.allclose(n, want, rtol=(D // 32 + 2) * 2 ** -24, atol=0)   # fp32 lane sums of D/32 squares
     op = tok.operand.float().cpu().numpy()
     assert np.array_equal(op, workloads.round_bf16(C))
     st = tok.level_stats.cpu().numpy()
