@@ -56,32 +56,42 @@ constexpr int BM = 128;       // rows per tile (TMEM lanes)
 constexpr int BN = 256;       // codewords per tile (UMMA N)
 constexpr int BK = 64;        // bf16 elements per k-block = one 128-byte swizzle row
 constexpr int UK = 16;        // K of one kind::f16 UMMA
-constexpr int NSTAGE = 4;
 constexpr int TOPK = 8;
 constexpr int MAX_SLOTS = 8;  // partial lists per row tile (bounds the rescore merge)
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
+// Norm term of the distance, folded into the GEMM as one extra K=16 step: A_aug rows are
+// (1, 1, 1, 0, ..., 0) and B_aug row j holds ||c_j||^2 / 2 split into three bf16 parts, so the
+// accumulator gets ||c_j||^2 / 2 on top of -r~.c~_j (the main steps negate A).  Both aug tiles
+// are K-major without swizzle: 8-row x 16-byte core matrices.
+constexpr int AUG_A_BYTES = (BM / 8) * 256;       // row groups 256 B apart, K halves 128 B apart
+constexpr int AUG_B_BYTES = (BN / 8) * 128 + 128;  // K half 1 aliases the next group (A's half 1 is 0)
+constexpr uint16_t BF16_ONE = 0x3F80;
+constexpr uint16_t BF16_BIG = 0x7F7F;  // largest finite bf16: codeword columns past K
 
 __device__ __forceinline__ float inf_f() { return __int_as_float(0x7f800000); }
 __device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
 
 // Thread organisation of the distance-GEMM block: EPI epilogue warps (EPI/4 column groups x 4
-// TMEM lane quadrants), then one TMA producer warp and one MMA-issuer warp.
+// TMEM lane quadrants), then the TMA producer warp, the MMA-issuer warp and the norm-split warp.
 template <int EPI>
 struct GemmCfg {
   static constexpr int GROUPS = EPI / 4;
   static constexpr int COLS = BN / GROUPS;  // columns of a tile one epilogue thread scans
   static constexpr int CHUNKS = COLS / 32;
   static constexpr int EPI_THREADS = EPI * 32;
-  static constexpr int THREADS = EPI_THREADS + 64;
+  static constexpr int THREADS = EPI_THREADS + 96;
   static constexpr int PRODUCER = EPI;
   static constexpr int ISSUER = EPI + 1;
-  static constexpr int NORM_OFF = NSTAGE * STAGE_BYTES;                  // 2 x 256 fp32 norms
-  static constexpr int MERGE_OFF = NORM_OFF + 2 * BN * 4;                // (GROUPS-1) x 128 x 8 x 8 B
+  static constexpr int SPLITTER = EPI + 2;
+  static constexpr int NSTAGE = EPI >= 16 ? 3 : 4;
+  static constexpr int AUG_A_OFF = NSTAGE * STAGE_BYTES;
+  static constexpr int AUG_B_OFF = AUG_A_OFF + AUG_A_BYTES;                // 2 slots
+  static constexpr int MERGE_OFF = AUG_B_OFF + 2 * AUG_B_BYTES;            // (GROUPS-1) x 128 x 8 x 8 B
   static constexpr int BAR_OFF = MERGE_OFF + (GROUPS - 1) * BM * TOPK * 8;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;                      // + barriers + alignment slack
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;                        // + barriers + alignment slack
 };
 
 struct GemmArgs {
@@ -93,7 +103,6 @@ struct GemmArgs {
   int Tc;     // codeword tiles
   int G;      // CTAs
   int maxs;   // partial-list slots per row tile
-  int bulk_norms;  // norms staged by bulk copy (K % 4 == 0)
   float2 *cand;
   int32_t *status;
 };
@@ -123,22 +132,29 @@ __device__ __forceinline__ void topk_insert(float (&bd)[TOPK], int (&bi)[TOPK], 
   }
 }
 
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const uint16_t *>(&b);
+}
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
 template <int EPI>
 __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     dist_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs a) {
   using C = GemmCfg<EPI>;
+  constexpr int NSTAGE = C::NSTAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *nslot = reinterpret_cast<float *>(smem + C::NORM_OFF);
+  uint8_t *aug_a = smem + C::AUG_A_OFF;
+  uint8_t *aug_b = smem + C::AUG_B_OFF;
   float2 *mbuf = reinterpret_cast<float2 *>(smem + C::MERGE_OFF);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
   uint64_t *empty = full + NSTAGE;
   uint64_t *tfull = empty + NSTAGE;
   uint64_t *tempty = tfull + 2;
-  uint64_t *nfull = tempty + 2;
-  uint64_t *nempty = nfull + 2;
-  uint64_t *mready = nempty + 2;
+  uint64_t *afull = tempty + 2;
+  uint64_t *mready = afull + 2;
   uint64_t *mdone = mready + 1;
   uint64_t *mma_done = mdone + 1;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
@@ -159,8 +175,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::EPI_THREADS);
-      mbar_init(&nfull[b], 1);
-      mbar_init(&nempty[b], C::EPI_THREADS);
+      mbar_init(&afull[b], 32);
     }
     mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
     mbar_init(mdone, 128);
@@ -169,6 +184,14 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     *never = 0;
     fence_mbar_init();
   }
+  // constant aug tiles: A_aug rows (1,1,1,0,...) and zeros everywhere else
+  for (int i = threadIdx.x; i < (AUG_A_BYTES + 2 * AUG_B_BYTES) / 16; i += blockDim.x) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (i < AUG_A_BYTES / 16 && ((i * 16) % 256) < 128)  // K half 0 of a row: elements 0..2 are one
+      v = make_uint4(BF16_ONE | (static_cast<uint32_t>(BF16_ONE) << 16), BF16_ONE, 0, 0);
+    reinterpret_cast<uint4 *>(aug_a)[i] = v;
+  }
+  fence_proxy_async_smem();
   if (warp == C::ISSUER) {
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
@@ -187,21 +210,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       uint32_t ph = 0;
       int64_t issued = 0;
       bool ok = true;
-      int64_t i = 0;
-      for (int64_t u = u0; u < u1 && ok; ++u, ++i) {
+      for (int64_t u = u0; u < u1 && ok; ++u) {
         const int64_t rt = u / a.Tc;
         const int ct = static_cast<int>(u - rt * a.Tc);
-        if (a.bulk_norms) {
-          const int slot = static_cast<int>(i & 1);
-          if (!mbar_wait(&nempty[slot], static_cast<uint32_t>((i >> 1) & 1) ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int nvalid = min(BN, a.K - ct * BN);  // a multiple of 4 when bulk_norms
-          mbar_arrive_expect_tx(&nfull[slot], static_cast<uint32_t>(nvalid * 4));
-          bulk_load(nslot + slot * BN, a.norms + static_cast<int64_t>(ct) * BN, static_cast<uint32_t>(nvalid * 4),
-                    &nfull[slot]);
-        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
@@ -232,16 +243,54 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
           }
           mbar_wait(&full[back], p, never);
         }
-        if (a.bulk_norms && i > 0) {
-          for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
-            mbar_wait(&nfull[j & 1], static_cast<uint32_t>((j >> 1) & 1), never);
-        }
       }
+    }
+  } else if (warp == C::SPLITTER) {
+    // ------------------------------------------------------------ norm split -> B_aug tiles
+    int64_t i = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1; ++u, ++i) {
+      const int slot = static_cast<int>(i & 1);
+      const int ct = static_cast<int>(u - (u / a.Tc) * a.Tc);
+      const int c0 = ct * BN + lane * 8;  // this lane fills row group `lane` (8 codewords)
+      float h[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) h[j] = c0 + j < a.K ? 0.5f * __ldg(a.norms + c0 + j) : 0.f;
+      // the slot is free once the MMAs of the unit two back (same slot) have completed
+      bool got = i < 2 || mbar_wait(&tfull[slot], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(aug_b + slot * AUG_B_BYTES + lane * 128);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint16_t h1, h2 = 0, h3 = 0;
+        if (c0 + j < a.K) {
+          h1 = bf16_bits_rn(h[j]);
+          const float r1 = h[j] - bf16_bits_to_float(h1);  // exact
+          h2 = bf16_bits_rn(r1);
+          const float r2 = r1 - bf16_bits_to_float(h2);    // exact
+          h3 = bf16_bits_rn(r2);
+        } else {
+          h1 = BF16_BIG;
+        }
+        dst[j] = make_uint4(h1 | (static_cast<uint32_t>(h2) << 16), h3, 0, 0);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&afull[slot]);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(a.status, RVQ_ERR_TIMEOUT);
     }
   } else if (warp == C::ISSUER) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc_main = idesc_bf16_f32(BM, BN, true);  // accumulates -r~.c~
+      constexpr uint32_t idesc_aug = idesc_bf16_f32(BM, BN, false);  // + ||c||^2 / 2
+      const uint64_t adesc_aug = sdesc_k_noswizzle(smem_u32(aug_a), 128, 256);
       int s = 0;
       uint32_t ph = 0;
       int64_t i = 0;
@@ -249,12 +298,13 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       for (int64_t u = u0; u < u1 && ok; ++u, ++i) {
         const int buf = static_cast<int>(i & 1);
         const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
-        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag) || !mbar_wait(&afull[buf], tph, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
+        umma_f16(dt, adesc_aug, sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128), idesc_aug, 0u);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
@@ -267,7 +317,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k)
             umma_f16(dt, ad + static_cast<uint64_t>(k * UK * 2 / 16), bd + static_cast<uint64_t>(k * UK * 2 / 16),
-                     idesc, (kb | k) != 0 ? 1u : 0u);
+                     idesc_main, 1u);
           umma_commit(&empty[s]);
           if (++s == NSTAGE) {
             s = 0;
@@ -286,6 +336,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue: running top-8
+    // TMEM holds half the shifted distance, ||c||^2/2 - r~.c~ = d~/2; lists keep d~/2 and are
+    // doubled (exactly) when written out.
     const int quad = warp & 3;
     const int grp = warp >> 2;
     const int row_in_tile = quad * 32 + lane;
@@ -332,7 +384,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
           float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK);
 #pragma unroll
           for (int t = 0; t < TOPK; t += 2)
-            out[t / 2] = make_float4(bd[t], __int_as_float(bi[t]), bd[t + 1], __int_as_float(bi[t + 1]));
+            out[t / 2] =
+                make_float4(2.f * bd[t], __int_as_float(bi[t]), 2.f * bd[t + 1], __int_as_float(bi[t + 1]));
         }
       }
       return true;
@@ -355,8 +408,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       }
       const int buf = static_cast<int>(i & 1);
       const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
-      bool got = mbar_wait(&tfull[buf], tph, abort_flag);
-      if (got && a.bulk_norms) got = mbar_wait(&nfull[buf], tph, abort_flag);
+      const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
@@ -377,37 +429,28 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         }
         const int c0 = col0 + ct0;
         float d[32];
-        if (a.bulk_norms && ct0 + 32 <= nvalid) {
-          const float4 *np = reinterpret_cast<const float4 *>(nslot + buf * BN + ct0);
+        if (ct0 + 32 <= nvalid) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 nn = np[j];
-            d[4 * j + 0] = fmaf(-2.f, __uint_as_float(v[4 * j + 0]), nn.x);
-            d[4 * j + 1] = fmaf(-2.f, __uint_as_float(v[4 * j + 1]), nn.y);
-            d[4 * j + 2] = fmaf(-2.f, __uint_as_float(v[4 * j + 2]), nn.z);
-            d[4 * j + 3] = fmaf(-2.f, __uint_as_float(v[4 * j + 3]), nn.w);
-          }
+          for (int j = 0; j < 32; ++j) d[j] = __uint_as_float(v[j]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            d[j] = (ct0 + j < nvalid) ? fmaf(-2.f, __uint_as_float(v[j]), __ldg(a.norms + c0 + j)) : inf_f();
+          for (int j = 0; j < 32; ++j) d[j] = (ct0 + j < nvalid) ? __uint_as_float(v[j]) : inf_f();
         }
-        // chunk minimum as a tree (short dependency chain)
-        float m16[16];
+        // chunk minimum as a tree of 3-input minima (short dependency chain)
+        float m11[11];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) m16[j] = fminf(d[j], d[j + 16]);
-#pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-          for (int j = 0; j < w; ++j) m16[j] = fminf(m16[j], m16[j + w]);
-        if (__any_sync(0xffffffffu, m16[0] < bd[TOPK - 1])) {
+        for (int j = 0; j < 10; ++j) m11[j] = fmin3(d[3 * j], d[3 * j + 1], d[3 * j + 2]);
+        m11[10] = fminf(d[30], d[31]);
+        const float m4a = fmin3(m11[0], m11[1], m11[2]), m4b = fmin3(m11[3], m11[4], m11[5]);
+        const float m4c = fmin3(m11[6], m11[7], m11[8]), m4d = fminf(m11[9], m11[10]);
+        const float m = fminf(fmin3(m4a, m4b, m4c), m4d);
+        if (__any_sync(0xffffffffu, m < bd[TOPK - 1])) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (__any_sync(0xffffffffu, d[j] < bd[TOPK - 1])) topk_insert(bd, bi, d[j], c0 + j);
           }
         }
       }
-      if (a.bulk_norms) mbar_arrive(&nempty[buf]);
     }
     if (ok && cur_rt >= 0 && !flush(cur_rt)) ok = false;
     if (!ok) {
@@ -531,11 +574,14 @@ struct RowArgs {
 
 __device__ __forceinline__ float error_bound(const float *st, float2 rs, int D) {
   const float cmax = st[0], dcmax = st[1], cqmax = st[2], nmax = st[3];
-  const float gamma = static_cast<float>(D + 16) * 2.384185791015625e-07f;  // 2^-22
+  // fp32 accumulation of D products and the three norm parts (truncation allowed)
+  const float gamma = static_cast<float>(D + 32) * 2.384185791015625e-07f;  // (D+32) 2^-22
   // norms: fp32 lane sums of ceil(D/32) squares combined in fp64, then rounded to fp32
   const float norm_err = static_cast<float>(D / 32 + 2) * 5.9604644775390625e-08f;  // (D/32+2) 2^-24
-  const float e = norm_err * nmax + 2.f * (rs.x * cmax + rs.y * dcmax) + 2.f * gamma * rs.y * cqmax +
-                  1.1920928955078125e-07f * (nmax + 2.f * rs.y * cqmax);
+  const float e = norm_err * nmax                                   // n vs ||c||^2
+                  + 2.f * (rs.x * cmax + rs.y * dcmax)              // bf16 rounding of r and c
+                  + 2.f * gamma * (rs.y * cqmax + 0.51f * nmax)     // tensor-core accumulation
+                  + 1.1920928955078125e-07f * nmax;                 // three-part bf16 split of n/2
   return 1.01f * e;
 }
 
@@ -923,7 +969,6 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ga.cand = cand;
     ga.status = status;
     profile_begin(s);
-    ga.bulk_norms = (K % 4) == 0 ? 1 : 0;
     launch_gemm(epi, p.G, s, tmA, tmB, ga);
     profile_end(s);
     note_launch();
