@@ -119,6 +119,35 @@ RVQ_API int rvq_encode(const void *features, int f_dtype, int64_t N, int D,
                void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
+ * rvq_encode_noalloc -- rvq_encode for callers that cannot allocate device memory.
+ * No counterpart in the pages: this is a deployment variant of rvq_encode.
+ *
+ * Some callers may not call cudaMalloc (or any allocating routine) at the point where they
+ * tokenize: code running under a framework that owns all device memory through its own pool,
+ * latency-critical serving loops that must not allocate (cudaMalloc can synchronize the
+ * device), or plugin hosts that hand out no workspace.  This entry point takes the same
+ * arguments as rvq_encode except the workspace: its scratch lives in a statically sized
+ * device array compiled into librvq.so, RVQ_NOALLOC_SCRATCH_BYTES bytes, which every GPU
+ * that loads the library holds until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - Sizes whose rvq_encode_workspace_size exceeds RVQ_NOALLOC_SCRATCH_BYTES are rejected with
+ *     RVQ_ERR_WORKSPACE before anything is enqueued (use rvq_encode with a workspace instead).
+ *   - The first call on a device looks up the scratch array's device address with that device
+ *     current (once per device); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (the kernels
+ *     initialise everything they read).  Calls that overlap on the GPU (different streams,
+ *     or threads) race on it: serialise them.
+ * Results are identical to rvq_encode with the same inputs.
+ */
+#define RVQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+RVQ_API int rvq_encode_noalloc(const void *features, int f_dtype, int64_t N, int D,
+                       const void *codebooks, int cb_dtype, const void *cb_operand,
+                       const float *norms, const float *level_stats, int L, int K,
+                       const int64_t *offsets, int64_t B,
+                       int32_t *ids, float *residual, float *recon, int32_t *fallbacks,
+                       int32_t *status, void *stream);
+
+/*
  * rvq_decode -- gather-sum de-tokenizer input (blog, Figure 1): recon[n] = sum_l C_l[ids[n,l]],
  * fp32 accumulation in ascending l.
  *   ids      [N, L] int32;  codebooks [L, K, D] in cb_dtype;  recon [N, D] fp32 out

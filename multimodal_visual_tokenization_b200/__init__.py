@@ -26,7 +26,9 @@ STATUS = {0: "RVQ_OK", -1: "RVQ_ERR_ARG", -2: "RVQ_ERR_UNSUPPORTED", -3: "RVQ_ER
           -4: "RVQ_ERR_CUDA", -5: "RVQ_ERR_ID_RANGE", -6: "RVQ_ERR_TIMEOUT"}
 
 EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
-           "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read")
+           "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read",
+           "rvq_encode_noalloc")
+RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _lib = None
 _lock = threading.Lock()
@@ -56,6 +58,8 @@ def load(path: str | None = None):
         lib.rvq_encode.argtypes = [vp, i32, i64, i32, vp, i32, vp, vp, vp, i32, i32, vp, i64,
                                    vp, vp, vp, vp, vp, sz, vp, vp]
         lib.rvq_decode.argtypes = [vp, i64, i32, vp, i32, i32, i32, vp, vp, vp]
+        lib.rvq_encode_noalloc.argtypes = [vp, i32, i64, i32, vp, i32, vp, vp, vp, i32, i32, vp, i64,
+                                           vp, vp, vp, vp, vp, vp]
         lib.rvq_status_str.argtypes = [i32]
         lib.rvq_status_str.restype = ctypes.c_char_p
         lib.rvq_launch_count.argtypes = []
@@ -63,7 +67,7 @@ def load(path: str | None = None):
         lib.rvq_profile_enable.argtypes = [i32]
         lib.rvq_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
-                   "rvq_profile_enable", "rvq_profile_read"):
+                   "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -121,6 +125,16 @@ def rvq_encode(features, f_dtype, N, D, codebooks, cb_dtype, cb_operand, norms, 
                              _ptr(norms), _ptr(level_stats), L, K, _ptr(offsets), B, _ptr(ids),
                              _ptr(residual), _ptr(recon), _ptr(fallbacks), _ptr(workspace),
                              workspace_bytes, _ptr(status), _stream(stream))
+
+
+def rvq_encode_noalloc(features, f_dtype, N, D, codebooks, cb_dtype, cb_operand, norms, level_stats, L, K,
+                       offsets, B, ids, residual, recon, fallbacks, status, stream=None):
+    """rvq_encode without a workspace argument, for callers that cannot allocate device memory:
+    the library's own statically sized scratch array (RVQ_NOALLOC_SCRATCH_BYTES) is used."""
+    return load().rvq_encode_noalloc(_ptr(features), f_dtype, N, D, _ptr(codebooks), cb_dtype,
+                                     _ptr(cb_operand), _ptr(norms), _ptr(level_stats), L, K, _ptr(offsets),
+                                     B, _ptr(ids), _ptr(residual), _ptr(recon), _ptr(fallbacks),
+                                     _ptr(status), _stream(stream))
 
 
 def rvq_decode(ids, N, L, codebooks, cb_dtype, K, D, recon, status, stream=None):

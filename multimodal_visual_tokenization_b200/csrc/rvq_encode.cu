@@ -1015,3 +1015,46 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   }
   return RVQ_OK;
 }
+
+// ---------------------------------------------------------------- encode without a caller workspace
+namespace rvq {
+namespace enc {
+
+// Scratch of rvq_encode_noalloc: one statically sized array per device, shared by all calls.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[RVQ_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device (host code cannot use the symbol
+// itself), looked up once per device with that device current.
+inline int noalloc_scratch(void **ptr) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RVQ_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RVQ_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return RVQ_OK;
+}
+
+}  // namespace enc
+}  // namespace rvq
+
+extern "C" int rvq_encode_noalloc(const void *features, int f_dtype, int64_t N, int D, const void *codebooks,
+                                  int cb_dtype, const void *cb_operand, const float *norms, const float *level_stats,
+                                  int L, int K, const int64_t *offsets, int64_t B, int32_t *ids, float *residual,
+                                  float *recon, int32_t *fallbacks, int32_t *status, void *stream) {
+  size_t need = 0;
+  int st = rvq_encode_workspace_size(N, D, L, K, &need);
+  if (st != RVQ_OK) return st;
+  if (need > RVQ_NOALLOC_SCRATCH_BYTES) return RVQ_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  st = rvq::enc::noalloc_scratch(&scratch);
+  if (st != RVQ_OK) return st;
+  return rvq_encode(features, f_dtype, N, D, codebooks, cb_dtype, cb_operand, norms, level_stats, L, K, offsets, B,
+                    ids, residual, recon, fallbacks, scratch, RVQ_NOALLOC_SCRATCH_BYTES, status, stream);
+}
