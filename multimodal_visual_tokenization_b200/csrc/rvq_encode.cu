@@ -72,6 +72,11 @@ constexpr uint16_t BF16_ONE = 0x3F80;
 constexpr uint16_t BF16_BIG = 0x7F7F;  // largest finite bf16: codeword columns past K
 
 __device__ __forceinline__ float inf_f() { return __int_as_float(0x7f800000); }
+constexpr float kPastK = 3.0e38f;  // key of a column past K (never a real half-distance)
+#ifndef RVQ_MERGE_LANES
+#define RVQ_MERGE_LANES 10
+#endif
+constexpr int kMergeLanes = RVQ_MERGE_LANES;  // lanes needing inserts that switch a chunk to the merge path
 __device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
 
 // Thread organisation of the distance-GEMM block: EPI epilogue warps (EPI/4 column groups x 4
@@ -129,6 +134,76 @@ __device__ __forceinline__ void topk_insert(float (&bd)[TOPK], int (&bi)[TOPK], 
   if (!c[0]) {
     bd[0] = x;
     bi[0] = ix;
+  }
+}
+
+// ---- branch-free top-8 of a 32-value chunk, used when many lanes of a warp need inserts at once.
+// Keys carry the chunk-local index in their 5 low mantissa bits (a relative perturbation below
+// 2^-18, covered by the certificate's error bound), so compare-exchanges are two min/max ops.
+__device__ __forceinline__ void cx(float &a, float &b) {
+  const float lo = fminf(a, b);
+  b = fmaxf(a, b);
+  a = lo;
+}
+// Batcher odd-even merge sort of 8 keys, ascending (19 compare-exchanges).
+__device__ __forceinline__ void sort8(float *v) {
+  cx(v[0], v[1]); cx(v[2], v[3]); cx(v[4], v[5]); cx(v[6], v[7]);
+  cx(v[0], v[2]); cx(v[1], v[3]); cx(v[4], v[6]); cx(v[5], v[7]);
+  cx(v[1], v[2]); cx(v[5], v[6]);
+  cx(v[0], v[4]); cx(v[1], v[5]); cx(v[2], v[6]); cx(v[3], v[7]);
+  cx(v[2], v[4]); cx(v[3], v[5]);
+  cx(v[1], v[2]); cx(v[3], v[4]); cx(v[5], v[6]);
+}
+// Smallest 8 of two ascending 8-lists, ascending: elementwise min against the reversed second
+// list gives a bitonic sequence, which three half-cleaner stages sort.
+__device__ __forceinline__ void merge8(float *a, const float *b) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) a[t] = fminf(a[t], b[7 - t]);
+  cx(a[0], a[4]); cx(a[1], a[5]); cx(a[2], a[6]); cx(a[3], a[7]);
+  cx(a[0], a[2]); cx(a[1], a[3]); cx(a[4], a[6]); cx(a[5], a[7]);
+  cx(a[0], a[1]); cx(a[2], a[3]); cx(a[4], a[5]); cx(a[6], a[7]);
+}
+__device__ __forceinline__ void cx_idx(float &a, float &b, int &ia, int &ib) {
+  const bool sw = b < a;
+  const float ta = a;
+  const int tia = ia;
+  a = sw ? b : a;
+  b = sw ? ta : b;
+  ia = sw ? ib : ia;
+  ib = sw ? tia : ib;
+}
+// Merge the chunk of 32 keys d[] (columns c0 + j, all finite) into the running list.
+__device__ __forceinline__ void topk_merge_chunk(float (&bd)[TOPK], int (&bi)[TOPK], const float (&d)[32], int c0) {
+  float k[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) k[j] = __uint_as_float((__float_as_uint(d[j]) & ~31u) | static_cast<uint32_t>(j));
+  sort8(k);
+  sort8(k + 8);
+  sort8(k + 16);
+  sort8(k + 24);
+  merge8(k, k + 8);
+  merge8(k + 16, k + 24);
+  merge8(k, k + 16);  // k[0..7]: the chunk's 8 smallest keys, ascending
+  float cv[TOPK];
+  int ci[TOPK];
+#pragma unroll
+  for (int t = 0; t < TOPK; ++t) {
+    const float q = k[TOPK - 1 - t];
+    const int qi = c0 + static_cast<int>(__float_as_uint(q) & 31u);
+    const bool keep = bd[t] <= q;
+    cv[t] = keep ? bd[t] : q;
+    ci[t] = keep ? bi[t] : qi;
+  }
+  cx_idx(cv[0], cv[4], ci[0], ci[4]); cx_idx(cv[1], cv[5], ci[1], ci[5]);
+  cx_idx(cv[2], cv[6], ci[2], ci[6]); cx_idx(cv[3], cv[7], ci[3], ci[7]);
+  cx_idx(cv[0], cv[2], ci[0], ci[2]); cx_idx(cv[1], cv[3], ci[1], ci[3]);
+  cx_idx(cv[4], cv[6], ci[4], ci[6]); cx_idx(cv[5], cv[7], ci[5], ci[7]);
+  cx_idx(cv[0], cv[1], ci[0], ci[1]); cx_idx(cv[2], cv[3], ci[2], ci[3]);
+  cx_idx(cv[4], cv[5], ci[4], ci[5]); cx_idx(cv[6], cv[7], ci[6], ci[7]);
+#pragma unroll
+  for (int t = 0; t < TOPK; ++t) {
+    bd[t] = cv[t];
+    bi[t] = ci[t];
   }
 }
 
@@ -383,6 +458,12 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
           const int slot = static_cast<int>(blockIdx.x) - cta_of_unit(rt * a.Tc, a.U, a.G);
           float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK);
 #pragma unroll
+          for (int t = 0; t < TOPK; ++t)
+            if (bi[t] >= a.K) {  // a past-K key kept only because the range had < 8 codewords
+              bd[t] = inf_f();
+              bi[t] = -1;
+            }
+#pragma unroll
           for (int t = 0; t < TOPK; t += 2)
             out[t / 2] =
                 make_float4(2.f * bd[t], __int_as_float(bi[t]), 2.f * bd[t + 1], __int_as_float(bi[t + 1]));
@@ -432,9 +513,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         if (ct0 + 32 <= nvalid) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) d[j] = __uint_as_float(v[j]);
-        } else {
+        } else {  // columns past K: a large finite key (the merge path packs indices into keys)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) d[j] = (ct0 + j < nvalid) ? __uint_as_float(v[j]) : inf_f();
+          for (int j = 0; j < 32; ++j) d[j] = (ct0 + j < nvalid) ? __uint_as_float(v[j]) : kPastK;
         }
         // chunk minimum as a tree of 3-input minima (short dependency chain)
         float m11[11];
@@ -444,7 +525,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         const float m4a = fmin3(m11[0], m11[1], m11[2]), m4b = fmin3(m11[3], m11[4], m11[5]);
         const float m4c = fmin3(m11[6], m11[7], m11[8]), m4d = fminf(m11[9], m11[10]);
         const float m = fminf(fmin3(m4a, m4b, m4c), m4d);
-        if (__any_sync(0xffffffffu, m < bd[TOPK - 1])) {
+        const unsigned need = __ballot_sync(0xffffffffu, m < bd[TOPK - 1]);
+        if (__popc(need) >= kMergeLanes) {
+          topk_merge_chunk(bd, bi, d, c0);  // many lanes: one branch-free merge for the warp
+        } else if (need) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (__any_sync(0xffffffffu, d[j] < bd[TOPK - 1])) topk_insert(bd, bi, d[j], c0 + j);
@@ -655,7 +739,9 @@ __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
   }
   const float T = warp_min_f(tl);
   const float dmin = warp_min_f(fminf(dv[0], dv[1]));
-  const float E = error_bound(a.stats, a.rowstat[n], a.D);
+  // + the index bits the chunk-merge path stores in candidate keys (relative change < 2^-18)
+  const float E = error_bound(a.stats, a.rowstat[n], a.D) +
+                  7.62939453125e-06f * (fabsf(dmin) + (T < 1e30f ? fabsf(T) : 0.f));  // 2^-17
 
   const float *r = a.R + n * a.D;
   double rr = 0.0;
