@@ -4,8 +4,8 @@
 One step = one pass of the whole path over one batch of synthetic native-resolution
 patch features, through the C ABI:
     rvq_build_norms (codeword norms + bf16 operand copy)
-    rvq_encode      (greedy RVQ: ids, fp32 residual and recon)
-    rvq_decode      (gather-sum of the produced ids)
+    rvq_encode      (greedy RVQ: ids and the fp32 final residual)
+    rvq_decode      (gather-sum of the produced ids: the reconstruction)
 Metric: tokens (feature vectors) per second, in millions.  `value` is measured with the
 inputs resident in HBM; `e2e` repeats it through the same calls with the features copied
 from pinned host memory every step and the ids + decoded recon copied back.
@@ -50,6 +50,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--rows", type=int, default=None, help="smaller N with the same recipe (profiling)")
+    p.add_argument("--gemm-events", choices=("timed", "separate"), default="timed",
+                   help="bracket distance-GEMM launches with events inside the timed steps, or in a "
+                        "separate pass of the same steps")
     return p.parse_args(argv)
 
 
@@ -259,7 +262,7 @@ def run_ours(args, rank, world, local_rank):
         check(mvt.rvq_build_norms(cb, tok.cb_dtype, L, K, D, tok.norms, tok.level_stats, tok.operand, stream),
               "rvq_build_norms")
         check(mvt.rvq_encode(xin, f_code, N, D, cb, tok.cb_dtype, tok.operand, tok.norms, tok.level_stats, L, K,
-                             off, B, ids, res, rec, fb, ws, ws_bytes, status, stream), "rvq_encode")
+                             off, B, ids, res, None, fb, ws, ws_bytes, status, stream), "rvq_encode")
         check(mvt.rvq_decode(ids if dec_ids is None else dec_ids, N, L, cb, tok.cb_dtype, K, D, rec2, status,
                              stream), "rvq_decode")
 
@@ -275,7 +278,8 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(gpu_index(local_rank)) as clk:
-        mvt.rvq_profile_enable(True)
+        in_timed = args.gemm_events == "timed"
+        mvt.rvq_profile_enable(in_timed)
         launches0 = mvt.rvq_launch_count()
         for k in range(args.steps):
             flush.zero_()
@@ -284,6 +288,12 @@ def run_ours(args, rank, world, local_rank):
             ends[k].record(stream)
         torch.cuda.synchronize(dev)
         launches = mvt.rvq_launch_count() - launches0
+        if not in_timed:  # the same steps again, GEMM launches bracketed by events
+            mvt.rvq_profile_enable(True)
+            for k in range(args.steps):
+                flush.zero_()
+                step(x)
+            torch.cuda.synchronize(dev)
         code, gemm_n, gemm_ms = mvt.rvq_profile_read()
         mvt.rvq_profile_enable(False)
     if world > 1:
@@ -305,7 +315,7 @@ def run_ours(args, rank, world, local_rank):
         check(mvt.rvq_build_norms(cb, tok.cb_dtype, L, K, D, tok.norms, tok.level_stats, tok.operand, stream), "")
         ev[1].record(stream)
         check(mvt.rvq_encode(x, f_code, N, D, cb, tok.cb_dtype, tok.operand, tok.norms, tok.level_stats, L, K,
-                             off, B, ids, res, rec, fb, ws, ws_bytes, status, stream), "")
+                             off, B, ids, res, None, fb, ws, ws_bytes, status, stream), "")
         ev[2].record(stream)
         check(mvt.rvq_decode(ids, N, L, cb, tok.cb_dtype, K, D, rec2, status, stream), "")
         ev[3].record(stream)
@@ -390,7 +400,8 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_label(spec), "N": N, "D": D, "L": L, "K": K,
-                   "step": "rvq_build_norms + rvq_encode(ids, residual, recon) + rvq_decode",
+                   "step": "rvq_build_norms + rvq_encode(ids, residual) + rvq_decode(ids -> recon)",
+                   "gemm_events": args.gemm_events,
                    "l2": "flushed between timed steps (512 MiB memset, outside the step events)",
                    "parallelism": f"replicas x{world}, rows independent, no data-path collective"},
         "roofline": roofline,

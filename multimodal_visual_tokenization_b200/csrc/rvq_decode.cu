@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t
                                                                   int L, const void *__restrict__ cb, int K,
                                                                   int D, float *__restrict__ recon,
                                                                   int32_t *status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t n = static_cast<int64_t>(blockIdx.x) * kDecodeWarps + (threadIdx.x >> 5);
   if (n >= N) return;  // whole warp
@@ -122,9 +124,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t
 }
 
 template <bool CB_BF16, int VEC>
-void launch_decode_t(const int32_t *ids, int64_t N, int L, const void *cb, int K, int D, float *recon,
-                     int32_t *status, cudaStream_t s, dim3 grid) {
-  decode_kernel<CB_BF16, VEC><<<grid, kDecodeWarps * 32, 0, s>>>(ids, N, L, cb, K, D, recon, status);
+cudaError_t launch_decode_t(const int32_t *ids, int64_t N, int L, const void *cb, int K, int D, float *recon,
+                            int32_t *status, cudaStream_t s, dim3 grid) {
+  return launch_pdl(decode_kernel<CB_BF16, VEC>, grid, dim3(kDecodeWarps * 32), 0, s, ids, N, L, cb, K, D, recon,
+                    status);
 }
 
 int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_dtype, int K, int D, float *recon,
@@ -135,16 +138,17 @@ int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_d
   const int gy = (D + 32 * vec - 1) / (32 * vec);
   if (gx > 0x7FFFFFFFLL || gy > 65535) return RVQ_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  cudaError_t e;
   if (cb_dtype == RVQ_BF16) {
     if (vec == 8)
-      launch_decode_t<true, 8>(ids, N, L, cb, K, D, recon, status, s, grid);
+      e = launch_decode_t<true, 8>(ids, N, L, cb, K, D, recon, status, s, grid);
     else
-      launch_decode_t<true, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
+      e = launch_decode_t<true, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
   } else {
-    launch_decode_t<false, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
+    e = launch_decode_t<false, 4>(ids, N, L, cb, K, D, recon, status, s, grid);
   }
   note_launch();
-  return check_launch();
+  return e == cudaSuccess ? RVQ_OK : RVQ_ERR_CUDA;
 }
 
 }  // namespace rvq

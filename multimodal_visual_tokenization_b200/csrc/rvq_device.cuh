@@ -18,6 +18,16 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: it lets the
+// next kernel in the stream start early (launch_dependents) and waits for the previous one to
+// finish and publish its memory (wait) before touching that kernel's outputs.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- addresses / timers
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -275,6 +275,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  griddep_launch_dependents();
+  griddep_wait();  // the residual operand and candidate buffers belong to the previous kernel until here
 
   if (warp == C::PRODUCER) {
     // ------------------------------------------------------------ TMA producer
@@ -617,6 +619,8 @@ __global__ void __launch_bounds__(256) init_kernel(const void *__restrict__ x, i
                                                    int32_t *__restrict__ fb_count, int L,
                                                    const int64_t *__restrict__ offsets, int64_t B,
                                                    int32_t *status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gtid < L) fb_count[gtid] = 0;
@@ -707,6 +711,8 @@ __device__ __forceinline__ void accept_row(const RowArgs &a, int64_t n, int id, 
 
 template <bool CB_BF16>
 __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (n >= a.N) return;
@@ -787,6 +793,8 @@ __global__ void __launch_bounds__(256) fallback_kernel(const RowArgs a) {
   __shared__ double wbest[8];
   __shared__ int wid[8];
   __shared__ int chosen;
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int count = *a.fb_count;
   for (int j = blockIdx.x; j < count; j += gridDim.x) {
@@ -956,14 +964,14 @@ inline bool gemm_attrs_ready(int epi) {
   return ok;
 }
 
-inline void launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                        const GemmArgs &ga) {
+inline cudaError_t launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                               const GemmArgs &ga) {
   if (epi == 4)
-    dist_topk_kernel<4><<<grid, GemmCfg<4>::THREADS, GemmCfg<4>::SMEM, s>>>(tmA, tmB, ga);
-  else if (epi == 16)
-    dist_topk_kernel<16><<<grid, GemmCfg<16>::THREADS, GemmCfg<16>::SMEM, s>>>(tmA, tmB, ga);
-  else
-    dist_topk_kernel<8><<<grid, GemmCfg<8>::THREADS, GemmCfg<8>::SMEM, s>>>(tmA, tmB, ga);
+    return launch_pdl(dist_topk_kernel<4>, dim3(grid), dim3(GemmCfg<4>::THREADS), GemmCfg<4>::SMEM, s, tmA, tmB, ga);
+  if (epi == 16)
+    return launch_pdl(dist_topk_kernel<16>, dim3(grid), dim3(GemmCfg<16>::THREADS), GemmCfg<16>::SMEM, s, tmA, tmB,
+                      ga);
+  return launch_pdl(dist_topk_kernel<8>, dim3(grid), dim3(GemmCfg<8>::THREADS), GemmCfg<8>::SMEM, s, tmA, tmB, ga);
 }
 
 }  // namespace enc
@@ -1026,14 +1034,15 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   {
     const int64_t threads = N * 32;
     const int64_t blocks = (threads + 255) / 256;
+    cudaError_t e;
     if (f_dtype == RVQ_BF16)
-      init_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(features, N, D, R, Rt, rowstat, fb_count, L,
-                                                                       offsets, B, status);
+      e = launch_pdl(init_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, features, N, D, R, Rt,
+                     rowstat, fb_count, L, offsets, B, status);
     else
-      init_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(features, N, D, R, Rt, rowstat, fb_count, L,
-                                                                        offsets, B, status);
+      e = launch_pdl(init_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, features, N, D, R,
+                     Rt, rowstat, fb_count, L, offsets, B, status);
     note_launch();
-    if ((st = check_launch()) != RVQ_OK) return st;
+    if (e != cudaSuccess) return RVQ_ERR_CUDA;
   }
 
   const int64_t row_blocks = (N * 32 + 255) / 256;
@@ -1055,10 +1064,10 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ga.cand = cand;
     ga.status = status;
     profile_begin(s);
-    launch_gemm(epi, p.G, s, tmA, tmB, ga);
+    const cudaError_t ge = launch_gemm(epi, p.G, s, tmA, tmB, ga);
     profile_end(s);
     note_launch();
-    if ((st = check_launch()) != RVQ_OK) return st;
+    if (ge != cudaSuccess) return RVQ_ERR_CUDA;
 
     RowArgs ra;
     ra.N = N;
@@ -1081,15 +1090,16 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ra.fb_count = fb_count + l;
     ra.status = status;
     ra.last = l == L - 1;
+    cudaError_t e1, e2;
     if (cb_dtype == RVQ_BF16) {
-      rescore_kernel<true><<<static_cast<unsigned>(row_blocks), 256, 0, s>>>(ra);
-      fallback_kernel<true><<<fb_blocks, 256, fb_smem, s>>>(ra);
+      e1 = launch_pdl(rescore_kernel<true>, dim3(static_cast<unsigned>(row_blocks)), dim3(256), 0, s, ra);
+      e2 = launch_pdl(fallback_kernel<true>, dim3(fb_blocks), dim3(256), fb_smem, s, ra);
     } else {
-      rescore_kernel<false><<<static_cast<unsigned>(row_blocks), 256, 0, s>>>(ra);
-      fallback_kernel<false><<<fb_blocks, 256, fb_smem, s>>>(ra);
+      e1 = launch_pdl(rescore_kernel<false>, dim3(static_cast<unsigned>(row_blocks)), dim3(256), 0, s, ra);
+      e2 = launch_pdl(fallback_kernel<false>, dim3(fb_blocks), dim3(256), fb_smem, s, ra);
     }
     note_launch(2);
-    if ((st = check_launch()) != RVQ_OK) return st;
+    if (e1 != cudaSuccess || e2 != cudaSuccess) return RVQ_ERR_CUDA;
   }
   if (fallbacks) {
     if (cudaMemcpyAsync(fallbacks, fb_count, sizeof(int32_t) * L, cudaMemcpyDeviceToDevice, s) != cudaSuccess)

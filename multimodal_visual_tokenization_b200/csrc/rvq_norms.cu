@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256) norms_kernel(const void *__restrict__ cb,
                                                     __nv_bfloat16 *__restrict__ cb_op) {
   __shared__ float wmax[8][RVQ_LEVEL_STATS];
   __shared__ int wlev[8];
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + warp;
@@ -134,12 +136,13 @@ extern "C" int rvq_build_norms(const void *codebooks, int cb_dtype, int L, int K
   const int64_t warps = static_cast<int64_t>(L) * K;
   const int64_t blocks = (warps + 7) / 8;
   if (blocks > 0x7FFFFFFFLL) return RVQ_ERR_UNSUPPORTED;
+  cudaError_t e;
   if (cb_dtype == RVQ_BF16)
-    norms_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(codebooks, L, K, D, norms, level_stats,
-                                                                      nullptr);
+    e = launch_pdl(norms_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, codebooks, L, K, D,
+                   norms, level_stats, static_cast<__nv_bfloat16 *>(nullptr));
   else
-    norms_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        codebooks, L, K, D, norms, level_stats, static_cast<__nv_bfloat16 *>(cb_operand));
+    e = launch_pdl(norms_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, codebooks, L, K, D,
+                   norms, level_stats, static_cast<__nv_bfloat16 *>(cb_operand));
   note_launch();
-  return check_launch();
+  return e == cudaSuccess ? RVQ_OK : RVQ_ERR_CUDA;
 }
