@@ -59,8 +59,6 @@ constexpr int UK = 16;        // K of one kind::f16 UMMA
 constexpr int TOPK = 8;
 constexpr int MAX_SLOTS = 8;  // partial lists per row tile (bounds the rescore merge)
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 // Norm term of the distance, folded into the GEMM as one extra K=16 step: A_aug rows are
 // (1, 1, 1, 0, ..., 0) and B_aug row j holds ||c_j||^2 / 2 split into three bf16 parts, so the
@@ -76,12 +74,14 @@ constexpr float kPastK = 3.0e38f;  // key of a column past K (never a real half-
 #ifndef RVQ_MERGE_LANES
 #define RVQ_MERGE_LANES 10
 #endif
-constexpr int kMergeLanes = RVQ_MERGE_LANES;  // lanes needing inserts that switch a chunk to the merge path
+constexpr int kMergeLanes = RVQ_MERGE_LANES;  // lanes needing inserts that switch a chunk to merging
 __device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
 
 // Thread organisation of the distance-GEMM block: EPI epilogue warps (EPI/4 column groups x 4
 // TMEM lane quadrants), then the TMA producer warp, the MMA-issuer warp and the norm-split warp.
-template <int EPI>
+// PAIR: the block is one CTA of a 2-CTA cluster that shares a 256-row x 256-codeword tile
+// (tcgen05 cta_group::2, M=256): each CTA loads its own 128 rows and 128 of the 256 codewords.
+template <int EPI, bool PAIR>
 struct GemmCfg {
   static constexpr int GROUPS = EPI / 4;
   static constexpr int COLS = BN / GROUPS;  // columns of a tile one epilogue thread scans
@@ -91,8 +91,10 @@ struct GemmCfg {
   static constexpr int PRODUCER = EPI;
   static constexpr int ISSUER = EPI + 1;
   static constexpr int SPLITTER = EPI + 2;
-  static constexpr int NSTAGE = EPI >= 16 ? 3 : 4;
-  static constexpr int AUG_A_OFF = NSTAGE * STAGE_BYTES;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // codeword rows this CTA loads per tile
+  static constexpr int STAGE = A_BYTES + B_ROWS * BK * 2;
+  static constexpr int NSTAGE = PAIR ? (EPI >= 16 ? 5 : 6) : (EPI >= 16 ? 3 : 4);
+  static constexpr int AUG_A_OFF = NSTAGE * STAGE;
   static constexpr int AUG_B_OFF = AUG_A_OFF + AUG_A_BYTES;                // 2 slots
   static constexpr int MERGE_OFF = AUG_B_OFF + 2 * AUG_B_BYTES;            // (GROUPS-1) x 128 x 8 x 8 B
   static constexpr int BAR_OFF = MERGE_OFF + (GROUPS - 1) * BM * TOPK * 8;
@@ -110,7 +112,10 @@ struct GemmArgs {
   int maxs;   // partial-list slots per row tile
   float2 *cand;
   int32_t *status;
+  int32_t *zero_counter;  // set to 0 by the first thread (the level's fallback counter), or null
 };
+// Units are (row tile, codeword tile) pairs; a row tile is 128 rows, or 256 for CTA pairs, and the
+// U units are split into G contiguous ranges, one per CTA (or per CTA pair).
 
 // CTA that owns unit u when U units are split into G contiguous ranges [cU/G, (c+1)U/G).
 __host__ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t U, int G) {
@@ -213,11 +218,11 @@ __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
 }
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
-template <int EPI>
-__global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
+template <int EPI, bool PAIR>
+__global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
     dist_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs a) {
-  using C = GemmCfg<EPI>;
+  using C = GemmCfg<EPI, PAIR>;
   constexpr int NSTAGE = C::NSTAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -238,9 +243,12 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.U / a.G;
-  const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * a.U / a.G;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
+  const int64_t cid = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  const int64_t u0 = cid * a.U / a.G;
+  const int64_t u1 = (cid + 1) * a.U / a.G;
   const int KB = a.D / BK;
+  constexpr int UNIT_ROWS = PAIR ? 2 * BM : BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -249,8 +257,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EPI_THREADS);
-      mbar_init(&afull[b], 32);
+      mbar_init(&tempty[b], (PAIR ? 2 : 1) * C::EPI_THREADS);
+      mbar_init(&afull[b], PAIR ? 64 : 32);
     }
     mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
     mbar_init(mdone, 128);
@@ -268,15 +276,28 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
   }
   fence_proxy_async_smem();
   if (warp == C::ISSUER) {
-    tmem_alloc(tmem_holder, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_holder, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the leader's barriers as seen from either CTA of the pair
+  const uint32_t full_l = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+  const uint32_t tempty_l = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
+  const uint32_t afull_l = PAIR ? mapa_shared(smem_u32(afull), 0) : 0u;
   griddep_launch_dependents();
   griddep_wait();  // the residual operand and candidate buffers belong to the previous kernel until here
+  if (a.zero_counter && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_counter = 0;
 
   if (warp == C::PRODUCER) {
     // ------------------------------------------------------------ TMA producer
@@ -290,15 +311,23 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       for (int64_t u = u0; u < u1 && ok; ++u) {
         const int64_t rt = u / a.Tc;
         const int ct = static_cast<int>(u - rt * a.Tc);
+        const int32_t row0 = static_cast<int32_t>(rt * UNIT_ROWS + rank * BM);
+        const int32_t cw0 = ct * BN + static_cast<int32_t>(rank) * C::B_ROWS;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          uint8_t *sa = smem + s * STAGE_BYTES;
-          tma_load_2d(&tmA, &full[s], sa, kb * BK, static_cast<int32_t>(rt * BM));
-          tma_load_2d(&tmB, &full[s], sa + A_BYTES, kb * BK, ct * BN);
+          uint8_t *sa = smem + s * C::STAGE;
+          if constexpr (PAIR) {  // both CTAs' bytes complete the leader's barrier
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
+            tma_load_2d_pair(&tmA, full_l + s * 8, sa, kb * BK, row0);
+            tma_load_2d_pair(&tmB, full_l + s * 8, sa + A_BYTES, kb * BK, cw0);
+          } else {
+            mbar_arrive_expect_tx(&full[s], C::STAGE);
+            tma_load_2d(&tmA, &full[s], sa, kb * BK, row0);
+            tma_load_2d(&tmB, &full[s], sa + A_BYTES, kb * BK, cw0);
+          }
           ++issued;
           if (++s == NSTAGE) {
             s = 0;
@@ -309,8 +338,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       if (!ok) {
         *abort_flag = 1;
         set_status(a.status, RVQ_ERR_TIMEOUT);
-        // no bulk copy may still be landing in shared memory when the block exits
-        const int64_t pending = issued < NSTAGE ? issued : NSTAGE;
+        // no bulk copy may still be landing in shared memory when the block exits (a pair's
+        // bytes are counted on the leader's barriers, so the leader drains for both)
+        const int64_t pending = (PAIR && rank != 0) ? 0 : (issued < NSTAGE ? issued : NSTAGE);
         for (int64_t j = 0; j < pending; ++j) {
           int back = s - 1 - static_cast<int>(j);
           uint32_t p = ph;
@@ -329,10 +359,12 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     for (int64_t u = u0; u < u1; ++u, ++i) {
       const int slot = static_cast<int>(i & 1);
       const int ct = static_cast<int>(u - (u / a.Tc) * a.Tc);
-      const int c0 = ct * BN + lane * 8;  // this lane fills row group `lane` (8 codewords)
+      constexpr int GROUPS_B = C::B_ROWS / 8;                       // row groups this CTA holds
+      const bool writer = lane < GROUPS_B;
+      const int c0 = ct * BN + static_cast<int>(rank) * C::B_ROWS + lane * 8;  // row group `lane`
       float h[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) h[j] = c0 + j < a.K ? 0.5f * __ldg(a.norms + c0 + j) : 0.f;
+      for (int j = 0; j < 8; ++j) h[j] = (writer && c0 + j < a.K) ? 0.5f * __ldg(a.norms + c0 + j) : 0.f;
       // the slot is free once the MMAs of the unit two back (same slot) have completed
       bool got = i < 2 || mbar_wait(&tfull[slot], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag);
       __syncwarp();
@@ -343,6 +375,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       uint4 *dst = reinterpret_cast<uint4 *>(aug_b + slot * AUG_B_BYTES + lane * 128);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
+        if (!writer) break;
         uint16_t h1, h2 = 0, h3 = 0;
         if (c0 + j < a.K) {
           h1 = bf16_bits_rn(h[j]);
@@ -356,17 +389,20 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         dst[j] = make_uint4(h1 | (static_cast<uint32_t>(h2) << 16), h3, 0, 0);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&afull[slot]);
+      if constexpr (PAIR)
+        mbar_arrive_cluster(afull_l + slot * 8);
+      else
+        mbar_arrive(&afull[slot]);
     }
     if (!ok) {
       *abort_flag = 1;
       set_status(a.status, RVQ_ERR_TIMEOUT);
     }
   } else if (warp == C::ISSUER) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_main = idesc_bf16_f32(BM, BN, true);  // accumulates -r~.c~
-      constexpr uint32_t idesc_aug = idesc_bf16_f32(BM, BN, false);  // + ||c||^2 / 2
+    // ------------------------------------------------------------ MMA issuer (the pair's leader)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc_main = idesc_bf16_f32(UNIT_ROWS, BN, true);  // accumulates -r~.c~
+      constexpr uint32_t idesc_aug = idesc_bf16_f32(UNIT_ROWS, BN, false);  // + ||c||^2 / 2
       const uint64_t adesc_aug = sdesc_k_noswizzle(smem_u32(aug_a), 128, 256);
       int s = 0;
       uint32_t ph = 0;
@@ -381,34 +417,51 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
-        umma_f16(dt, adesc_aug, sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128), idesc_aug, 0u);
+        const uint64_t bdesc_aug = sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128);
+        if constexpr (PAIR)
+          umma_f16_pair(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
+        else
+          umma_f16(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + s * C::STAGE);
           const uint64_t ad = sdesc_k128(sa);
           const uint64_t bd = sdesc_k128(sa + A_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            umma_f16(dt, ad + static_cast<uint64_t>(k * UK * 2 / 16), bd + static_cast<uint64_t>(k * UK * 2 / 16),
-                     idesc_main, 1u);
-          umma_commit(&empty[s]);
+          for (int k = 0; k < BK / UK; ++k) {
+            const uint64_t step = static_cast<uint64_t>(k * UK * 2 / 16);
+            if constexpr (PAIR)
+              umma_f16_pair(dt, ad + step, bd + step, idesc_main, 1u);
+            else
+              umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
+          }
+          if constexpr (PAIR)
+            umma_commit_pair_mc(&empty[s], 0x3);  // frees the stage in both CTAs
+          else
+            umma_commit(&empty[s]);
           if (++s == NSTAGE) {
             s = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[buf]);
+        if constexpr (PAIR)
+          umma_commit_pair_mc(&tfull[buf], 0x3);  // both CTAs' epilogues may read their TMEM
+        else
+          umma_commit(&tfull[buf]);
       }
       if (!ok) {
         *abort_flag = 1;
         set_status(a.status, RVQ_ERR_TIMEOUT);
       }
-      umma_commit(mma_done);
+      if constexpr (PAIR)
+        umma_commit_pair(mma_done);
+      else
+        umma_commit(mma_done);
       mbar_wait(mma_done, 0, never);
     }
   } else {
@@ -455,10 +508,11 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
       }
       ++nflush;
       if (grp == 0) {
-        const int64_t n = rt * BM + row_in_tile;
+        const int64_t rt128 = rt * (UNIT_ROWS / BM) + rank;  // this CTA's 128-row tile
+        const int64_t n = rt128 * BM + row_in_tile;
         if (n < a.N) {
-          const int slot = static_cast<int>(blockIdx.x) - cta_of_unit(rt * a.Tc, a.U, a.G);
-          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK);
+          const int slot = static_cast<int>(cid) - cta_of_unit(rt * a.Tc, a.U, a.G);
+          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt128 * a.maxs + slot) * BM + row_in_tile) * TOPK);
 #pragma unroll
           for (int t = 0; t < TOPK; ++t)
             if (bi[t] >= a.K) {  // a past-K key kept only because the range had < 8 codewords
@@ -508,7 +562,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
         tmem_ld_wait();
         if (ch == C::CHUNKS - 1) {
           tc_fence_before();
-          mbar_arrive(&tempty[buf]);
+          if constexpr (PAIR)
+            mbar_arrive_cluster(tempty_l + buf * 8);
+          else
+            mbar_arrive(&tempty[buf]);
         }
         const int c0 = col0 + ct0;
         float d[32];
@@ -546,11 +603,18 @@ __global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if constexpr (PAIR)
+    cluster_sync();  // neither CTA leaves while the leader's MMAs may still use its memory
+  else
+    __syncthreads();
   tc_fence_after();
   if (warp == C::ISSUER) {
     __syncwarp();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -613,7 +677,7 @@ __device__ __forceinline__ float2 write_operand_row(const float *r, __nv_bfloat1
 
 // r_0 = fp32(x), its bf16 operand copy and row statistics; also clears the fallback counters
 // and checks the packed-batch offsets.
-template <bool X_BF16>
+template <bool X_BF16, bool WRITE_R>
 __global__ void __launch_bounds__(256) init_kernel(const void *__restrict__ x, int64_t N, int D, float *__restrict__ R,
                                                    __nv_bfloat16 *__restrict__ Rt, float2 *__restrict__ rowstat,
                                                    int32_t *__restrict__ fb_count, int L,
@@ -632,20 +696,26 @@ __global__ void __launch_bounds__(256) init_kernel(const void *__restrict__ x, i
   }
   const int64_t n = gtid >> 5;
   if (n >= N) return;
-  float *r = R + n * D;
+  float e2 = 0.f, q2 = 0.f;
   for (int i = lane * 4; i < D; i += 128) {
     const float4 v = ld4<X_BF16>(x, n * D + i);
-    *reinterpret_cast<float4 *>(r + i) = v;
+    if constexpr (WRITE_R) *reinterpret_cast<float4 *>(R + n * D + i) = v;
+    float4 q;
+    store_bf16x4(Rt + n * D + i, v, &q);
+    const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+    e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+    q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
   }
-  __syncwarp();
-  const float2 st = write_operand_row(r, Rt + n * D, D, lane);
-  if (lane == 0) rowstat[n] = st;
+  e2 = warp_sum_f(e2);
+  q2 = warp_sum_f(q2);
+  if (lane == 0) rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
 }
 
 struct RowArgs {
   int64_t N;
   int D, K, L, l;
   int Tc, G, maxs;
+  int pair;  // units span 256 rows (CTA pairs) instead of 128
   int64_t U;
   const float2 *cand;
   float2 *rowstat;
@@ -658,7 +728,29 @@ struct RowArgs {
   int32_t *fb_count;     // this level's counter
   int32_t *status;
   int last;              // no operand copy needed after the last level
+  // register-resident path (D <= 1024)
+  const void *src;       // residual before this level: R, or the features at level 0
+  int32_t *fb_next;      // next level's fallback counter to clear, or null
+  const int64_t *offsets;  // checked at level 0, else null
+  int64_t B;
 };
+
+// Where a level's input residual comes from.
+enum RowSrc { SRC_R = 0, SRC_X_F32 = 1, SRC_X_BF16 = 2 };
+
+template <int SRC>
+__device__ __forceinline__ float4 ld_src4(const void *p, int64_t off) {
+  if constexpr (SRC == SRC_X_BF16) {
+    uint2 raw = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p) + off));
+    float2 x = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
+    float2 y = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
+    return make_float4(x.x, x.y, y.x, y.y);
+  } else if constexpr (SRC == SRC_X_F32) {
+    return __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off));
+  } else {  // the running residual, written by the previous level: no read-only cache
+    return *reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off);
+  }
+}
 
 __device__ __forceinline__ float error_bound(const float *st, float2 rs, int D) {
   const float cmax = st[0], dcmax = st[1], cqmax = st[2], nmax = st[3];
@@ -718,8 +810,9 @@ __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
   if (n >= a.N) return;
   const int64_t rt = n / BM;
   const int rin = static_cast<int>(n - rt * BM);
-  const int c0 = cta_of_unit(rt * a.Tc, a.U, a.G);
-  const int c1 = cta_of_unit(rt * a.Tc + a.Tc - 1, a.U, a.G);
+  const int64_t ut = a.pair ? (rt >> 1) : rt;  // the unit row tile this 128-row tile belongs to
+  const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
+  const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
   const int ncand = (c1 - c0 + 1) * TOPK;
 
   float dv[2];
@@ -854,21 +947,306 @@ __global__ void __launch_bounds__(256) fallback_kernel(const RowArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- register-resident row kernels
+// One warp per row with the whole residual row in registers (NCH float4 per lane, D <= 128*NCH):
+// the candidate lists, the row and the winner's codeword are each read once, and the updated
+// residual, its bf16 operand copy and row statistics are written from registers.
+
+template <bool CB_BF16, int SRC, int NCH>
+__global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gtid == 0 && a.fb_next) *a.fb_next = 0;
+  if (a.offsets) {  // packed-batch bookkeeping: offsets[0] = 0, non-decreasing, offsets[B] = N
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t b = gtid; b < a.B; b += nthreads)
+      if (a.offsets[b] > a.offsets[b + 1]) set_status(a.status, RVQ_ERR_ARG);
+    if (gtid == 0 && (a.offsets[0] != 0 || a.offsets[a.B] != a.N)) set_status(a.status, RVQ_ERR_ARG);
+  }
+  const int64_t n = gtid >> 5;
+  if (n >= a.N) return;
+  const int64_t rt = n / BM;
+  const int rin = static_cast<int>(n - rt * BM);
+  const int64_t ut = a.pair ? (rt >> 1) : rt;
+  const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
+  const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
+  const int ncand = (c1 - c0 + 1) * TOPK;
+
+  // independent loads first: the residual row and the candidate lists
+  float4 rv[NCH];
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    rv[k] = i < a.D ? ld_src4<SRC>(a.src, n * a.D + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float dv[2];
+  int iv[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = lane + 32 * h;
+    dv[h] = inf_f();
+    iv[h] = -1;
+    if (e < ncand) {
+      const int slot = e / TOPK, t = e - slot * TOPK;
+      const float2 c = a.cand[((rt * a.maxs + slot) * BM + rin) * TOPK + t];
+      dv[h] = c.x;
+      iv[h] = __float_as_int(c.y);
+    }
+  }
+  float2 rs = make_float2(0.f, 0.f);
+  if constexpr (SRC != SRC_X_BF16) rs = a.rowstat[n];
+
+  // r is its own bf16 copy when it comes straight from bf16 features: e_r = 0, ||r~|| = ||r||
+  if constexpr (SRC == SRC_X_BF16) {
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) q += rv[k].x * rv[k].x + rv[k].y * rv[k].y + rv[k].z * rv[k].z + rv[k].w * rv[k].w;
+    rs = make_float2(0.f, __fsqrt_ru(1.0001f * warp_sum_f(q)));
+  }
+
+  float tl = inf_f();
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = lane + 32 * h;
+    if (e < ncand && (e % TOPK) == TOPK - 1) tl = fminf(tl, dv[h]);
+  }
+  const float T = warp_min_f(tl);
+  const float dmin = warp_min_f(fminf(dv[0], dv[1]));
+  const float E = error_bound(a.stats, rs, a.D) + 7.62939453125e-06f * (fabsf(dmin) + (T < 1e30f ? fabsf(T) : 0.f));
+  const float lim = dmin + 2.f * E;
+  const unsigned pm0 = __ballot_sync(0xffffffffu, iv[0] >= 0 && dv[0] <= lim);
+  const unsigned pm1 = __ballot_sync(0xffffffffu, iv[1] >= 0 && dv[1] <= lim);
+
+  int best_id = 0x7fffffff;
+  float4 cbest[NCH];
+  if (__popc(pm0) + __popc(pm1) == 1 && T - dmin > 2.f * E) {
+    // One candidate within 2E of the best score and every dropped score more than 2E above it:
+    // its true distance is below every other codeword's, so no exact rescore is needed.
+    best_id = pm0 ? __shfl_sync(0xffffffffu, iv[0], __ffs(pm0) - 1) : __shfl_sync(0xffffffffu, iv[1], __ffs(pm1) - 1);
+    const int64_t coff = (static_cast<int64_t>(a.l) * a.K + best_id) * a.D;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int i = lane * 4 + k * 128;
+      cbest[k] = i < a.D ? ld4<CB_BF16>(a.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else {
+    double rr = 0.0;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k)
+      rr += static_cast<double>(rv[k].x) * rv[k].x + static_cast<double>(rv[k].y) * rv[k].y +
+            static_cast<double>(rv[k].z) * rv[k].z + static_cast<double>(rv[k].w) * rv[k].w;
+    rr = warp_sum_d(rr);
+    double best = inf_d();
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) cbest[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      unsigned mask = h == 0 ? pm0 : pm1;
+      while (mask) {
+        const int srcl = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int id = __shfl_sync(0xffffffffu, iv[h], srcl);
+        const int64_t coff = (static_cast<int64_t>(a.l) * a.K + id) * a.D;
+        float4 c[NCH];
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          const int i = lane * 4 + k * 128;
+          c[k] = i < a.D ? ld4<CB_BF16>(a.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        double dd = 0.0;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          const double e0 = static_cast<double>(rv[k].x) - c[k].x, e1 = static_cast<double>(rv[k].y) - c[k].y;
+          const double e2 = static_cast<double>(rv[k].z) - c[k].z, e3 = static_cast<double>(rv[k].w) - c[k].w;
+          dd += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+        }
+        dd = warp_sum_d(dd);
+        if (dd < best || (dd == best && id < best_id)) {
+          best = dd;
+          best_id = id;
+#pragma unroll
+          for (int k = 0; k < NCH; ++k) cbest[k] = c[k];
+        }
+      }
+    }
+    const bool certified =
+        best_id != 0x7fffffff && (best - rr) < (static_cast<double>(T) - static_cast<double>(E));
+    if (!certified) {
+      if (lane == 0) {
+        const int pos = atomicAdd(a.fb_count, 1);
+        a.fb_list[pos] = static_cast<int32_t>(n);
+      }
+      return;
+    }
+  }
+  float e2 = 0.f, q2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    if (i >= a.D) break;
+    float4 v = rv[k];
+    v.x -= cbest[k].x;
+    v.y -= cbest[k].y;
+    v.z -= cbest[k].z;
+    v.w -= cbest[k].w;
+    *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
+    if (!a.last) {
+      float4 q;
+      store_bf16x4(a.Rt + n * a.D + i, v, &q);
+      const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+      e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+      q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+    }
+  }
+  if (!a.last) {
+    e2 = warp_sum_f(e2);
+    q2 = warp_sum_f(q2);
+    if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
+  }
+  if (lane == 0) a.ids[n * a.L + a.l] = best_id;
+}
+
+// Exact scan of all K codewords for the rows this level's rescore could not certify.
+template <bool CB_BF16, int SRC>
+__global__ void __launch_bounds__(256) fallback_fast_kernel(const RowArgs a) {
+  extern __shared__ double sr[];  // residual row widened to fp64
+  __shared__ double wbest[8];
+  __shared__ int wid[8];
+  __shared__ int chosen;
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int count = *a.fb_count;
+  for (int j = blockIdx.x; j < count; j += gridDim.x) {
+    const int64_t n = a.fb_list[j];
+    __syncthreads();
+    for (int i = threadIdx.x * 4; i < a.D; i += blockDim.x * 4) {
+      const float4 v = ld_src4<SRC>(a.src, n * a.D + i);
+      sr[i] = v.x;
+      sr[i + 1] = v.y;
+      sr[i + 2] = v.z;
+      sr[i + 3] = v.w;
+    }
+    __syncthreads();
+    double bd = inf_d();
+    int bk = 0x7fffffff;
+    for (int k = warp; k < a.K; k += 8) {
+      const int64_t coff = (static_cast<int64_t>(a.l) * a.K + k) * a.D;
+      double acc = 0.0;
+      for (int i = lane * 4; i < a.D; i += 128) {
+        const float4 c = ld4<CB_BF16>(a.cb, coff + i);
+        const double e0 = sr[i] - c.x, e1 = sr[i + 1] - c.y, e2 = sr[i + 2] - c.z, e3 = sr[i + 3] - c.w;
+        acc += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+      }
+      acc = warp_sum_d(acc);
+      if (acc < bd) {
+        bd = acc;
+        bk = k;
+      }
+    }
+    if (lane == 0) {
+      wbest[warp] = bd;
+      wid[warp] = bk;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double b = wbest[0];
+      int k = wid[0];
+      for (int w = 1; w < 8; ++w)
+        if (wbest[w] < b || (wbest[w] == b && wid[w] < k)) {
+          b = wbest[w];
+          k = wid[w];
+        }
+      chosen = k;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int id = chosen;
+      if (id < 0 || id >= a.K) {  // only reachable with non-finite inputs
+        if (lane == 0) {
+          a.ids[n * a.L + a.l] = -1;
+          set_status(a.status, RVQ_ERR_ARG);
+        }
+        continue;
+      }
+      const int64_t coff = (static_cast<int64_t>(a.l) * a.K + id) * a.D;
+      float e2 = 0.f, q2 = 0.f;
+      for (int i = lane * 4; i < a.D; i += 128) {
+        const float4 c = ld4<CB_BF16>(a.cb, coff + i);
+        const float4 v = make_float4(static_cast<float>(sr[i]) - c.x, static_cast<float>(sr[i + 1]) - c.y,
+                                     static_cast<float>(sr[i + 2]) - c.z, static_cast<float>(sr[i + 3]) - c.w);
+        *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
+        if (!a.last) {
+          float4 q;
+          store_bf16x4(a.Rt + n * a.D + i, v, &q);
+          const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+          e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+          q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+        }
+      }
+      if (!a.last) {
+        e2 = warp_sum_f(e2);
+        q2 = warp_sum_f(q2);
+        if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
+      }
+      if (lane == 0) a.ids[n * a.L + a.l] = id;
+    }
+  }
+}
+
+template <bool CB_BF16, int SRC>
+inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blocks, int fb_blocks, size_t fb_smem,
+                                    cudaStream_t s) {
+  cudaError_t e;
+  switch (nch) {
+    case 1: e = launch_pdl(rescore_fast_kernel<CB_BF16, SRC, 1>, dim3(row_blocks), dim3(256), 0, s, ra); break;
+    case 2: e = launch_pdl(rescore_fast_kernel<CB_BF16, SRC, 2>, dim3(row_blocks), dim3(256), 0, s, ra); break;
+    case 4: e = launch_pdl(rescore_fast_kernel<CB_BF16, SRC, 4>, dim3(row_blocks), dim3(256), 0, s, ra); break;
+    default: e = launch_pdl(rescore_fast_kernel<CB_BF16, SRC, 8>, dim3(row_blocks), dim3(256), 0, s, ra); break;
+  }
+  if (e != cudaSuccess) return e;
+  return launch_pdl(fallback_fast_kernel<CB_BF16, SRC>, dim3(fb_blocks), dim3(256), fb_smem, s, ra);
+}
+
 // ---------------------------------------------------------------- host plan
 
 struct Plan {
-  int64_t RT;
+  int64_t RT;  // 128-row tiles
   int Tc;
   int64_t U;
-  int G;
+  int G;       // CTAs, or CTA pairs when pair
   int maxs;
+  bool pair;
 };
 
-inline Plan make_plan(int64_t N, int K, int sms) {
+// CTA pairs (tcgen05 cta_group::2) halve the codeword traffic per SM.  Off unless RVQ_PAIR=1
+// (tuning knob): on the measured workloads the single-CTA kernel is not L2-bound.
+inline bool use_pairs(int64_t N) {
+  static int forced = [] {
+    const char *e = getenv("RVQ_PAIR");
+    return e ? (atoi(e) != 0 ? 1 : 0) : -1;
+  }();
+  return forced >= 0 ? forced == 1 : false;  // measured: no gain over single CTAs at D = 256, 1024
+}
+
+int resident_pair_clusters(int D);
+
+inline Plan make_plan(int64_t N, int K, int D, int sms) {
   Plan p;
+  p.pair = use_pairs(N);
+  if (p.pair) {
+    const int clusters = resident_pair_clusters(D);
+    if (clusters < 1)
+      p.pair = false;
+    else
+      sms = std::min(sms / 2, clusters);
+  }
   p.RT = (N + BM - 1) / BM;
   p.Tc = (K + BN - 1) / BN;
-  p.U = p.RT * p.Tc;
+  const int64_t unit_rows = p.pair ? 2 * BM : BM;
+  p.U = ((N + unit_rows - 1) / unit_rows) * p.Tc;
   // every CTA covers at least f = floor(U/G) units, so a row tile (Tc consecutive units) meets
   // at most 1 + ceil((Tc-1)/f) CTAs; keep that within the rescore warp's candidate capacity
   const int64_t slots_cap = MAX_SLOTS;
@@ -937,10 +1315,10 @@ inline bool make_map(CUtensorMap *m, const void *base, int64_t rows, int D, int 
 }
 
 
-template <int EPI>
+template <int EPI, bool PAIR>
 inline bool set_gemm_attr() {
-  return cudaFuncSetAttribute(dist_topk_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<EPI>::SMEM) == cudaSuccess;
+  return cudaFuncSetAttribute(dist_topk_kernel<EPI, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<EPI, PAIR>::SMEM) == cudaSuccess;
 }
 
 // Epilogue warps of the distance GEMM.  A short feature width gives little MMA time per tile to
@@ -959,19 +1337,75 @@ inline int epilogue_warps(int D) {
 inline bool gemm_attrs_ready(int epi) {
   static std::once_flag once;
   static bool ok = false;
-  std::call_once(once, [] { ok = set_gemm_attr<4>() && set_gemm_attr<8>() && set_gemm_attr<16>(); });
+  std::call_once(once, [] {
+    ok = set_gemm_attr<4, false>() && set_gemm_attr<8, false>() && set_gemm_attr<16, false>() &&
+         set_gemm_attr<4, true>() && set_gemm_attr<8, true>() && set_gemm_attr<16, true>();
+  });
   (void)epi;
   return ok;
 }
 
-inline cudaError_t launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                               const GemmArgs &ga) {
-  if (epi == 4)
-    return launch_pdl(dist_topk_kernel<4>, dim3(grid), dim3(GemmCfg<4>::THREADS), GemmCfg<4>::SMEM, s, tmA, tmB, ga);
-  if (epi == 16)
-    return launch_pdl(dist_topk_kernel<16>, dim3(grid), dim3(GemmCfg<16>::THREADS), GemmCfg<16>::SMEM, s, tmA, tmB,
-                      ga);
-  return launch_pdl(dist_topk_kernel<8>, dim3(grid), dim3(GemmCfg<8>::THREADS), GemmCfg<8>::SMEM, s, tmA, tmB, ga);
+template <int EPI, bool PAIR>
+inline cudaError_t launch_gemm_t(int groups, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                 const GemmArgs &ga) {
+  using C = GemmCfg<EPI, PAIR>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(groups * (PAIR ? 2 : 1));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, dist_topk_kernel<EPI, PAIR>, tmA, tmB, ga);
+}
+
+// Clusters of two GEMM CTAs that can be resident at once (an SM pair must share a GPC).
+template <int EPI>
+inline int max_pair_clusters() {
+  static int n = [] {
+    using C = GemmCfg<EPI, true>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, dist_topk_kernel<EPI, true>, &cfg) != cudaSuccess) clusters = 0;
+    return clusters;
+  }();
+  return n;
+}
+
+// Resident CTA-pair clusters for the epilogue width that feature width D selects.
+inline int resident_pair_clusters(int D) {
+  if (!gemm_attrs_ready(0)) return 0;
+  const int epi = epilogue_warps(D);
+  return epi == 4 ? max_pair_clusters<4>() : epi == 16 ? max_pair_clusters<16>() : max_pair_clusters<8>();
+}
+
+inline cudaError_t launch_gemm(int epi, bool pair, int groups, cudaStream_t s, const CUtensorMap &tmA,
+                               const CUtensorMap &tmB, const GemmArgs &ga) {
+  if (pair) {
+    if (epi == 4) return launch_gemm_t<4, true>(groups, s, tmA, tmB, ga);
+    if (epi == 16) return launch_gemm_t<16, true>(groups, s, tmA, tmB, ga);
+    return launch_gemm_t<8, true>(groups, s, tmA, tmB, ga);
+  }
+  if (epi == 4) return launch_gemm_t<4, false>(groups, s, tmA, tmB, ga);
+  if (epi == 16) return launch_gemm_t<16, false>(groups, s, tmA, tmB, ga);
+  return launch_gemm_t<8, false>(groups, s, tmA, tmB, ga);
 }
 
 }  // namespace enc
@@ -984,7 +1418,7 @@ extern "C" int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t 
   int sms = 0;
   int st = device_sm_count(&sms);
   if (st != RVQ_OK) return st;
-  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, sms);
+  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, sms);
   *bytes = enc::make_layout(N, D, p).total;
   return RVQ_OK;
 }
@@ -1012,7 +1446,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   int sms = 0;
   int st = device_sm_count(&sms);
   if (st != RVQ_OK) return st;
-  const Plan p = make_plan(N, K, sms);
+  const Plan p = make_plan(N, K, D, sms);
   const Layout w = make_layout(N, D, p);
   if (workspace_bytes < w.total) return RVQ_ERR_WORKSPACE;
 
@@ -1031,19 +1465,30 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   const int epi = epilogue_warps(D);
   if (!gemm_attrs_ready(epi)) return RVQ_ERR_CUDA;
 
-  {
+  // D <= 1024: register-resident row kernels; level 0 reads the features directly (bf16 features
+  // are their own tensor-core operand, so no initial copy at all).  Wider rows: the init kernel
+  // materialises the fp32 residual and the row kernels stream it.
+  const bool fast = D <= 1024;
+  const int nch = D <= 128 ? 1 : D <= 256 ? 2 : D <= 512 ? 4 : 8;
+  const bool x_is_operand = fast && f_dtype == RVQ_BF16;
+  if (!x_is_operand) {
     const int64_t threads = N * 32;
-    const int64_t blocks = (threads + 255) / 256;
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     cudaError_t e;
-    if (f_dtype == RVQ_BF16)
-      e = launch_pdl(init_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, features, N, D, R, Rt,
-                     rowstat, fb_count, L, offsets, B, status);
+    if (fast)  // only the level-0 operand copy and row statistics
+      e = launch_pdl(init_kernel<false, false>, dim3(blocks), dim3(256), 0, s, features, N, D, R, Rt, rowstat,
+                     fb_count, 0, static_cast<const int64_t *>(nullptr), int64_t(0), status);
+    else if (f_dtype == RVQ_BF16)
+      e = launch_pdl(init_kernel<true, true>, dim3(blocks), dim3(256), 0, s, features, N, D, R, Rt, rowstat,
+                     fb_count, L, offsets, B, status);
     else
-      e = launch_pdl(init_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, features, N, D, R,
-                     Rt, rowstat, fb_count, L, offsets, B, status);
+      e = launch_pdl(init_kernel<false, true>, dim3(blocks), dim3(256), 0, s, features, N, D, R, Rt, rowstat,
+                     fb_count, L, offsets, B, status);
     note_launch();
     if (e != cudaSuccess) return RVQ_ERR_CUDA;
   }
+  CUtensorMap tmX;
+  if (x_is_operand && !make_map(&tmX, features, N, D, BM)) return RVQ_ERR_CUDA;
 
   const int64_t row_blocks = (N * 32 + 255) / 256;
   const int fb_blocks = 2 * sms;
@@ -1051,7 +1496,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   for (int l = 0; l < L; ++l) {
     const size_t lvl = static_cast<size_t>(l) * K * D * 2;
     CUtensorMap tmB;
-    if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, BN)) return RVQ_ERR_CUDA;
+    if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, p.pair ? BN / 2 : BN)) return RVQ_ERR_CUDA;
     GemmArgs ga;
     ga.norms = norms + static_cast<size_t>(l) * K;
     ga.N = N;
@@ -1063,8 +1508,9 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ga.maxs = p.maxs;
     ga.cand = cand;
     ga.status = status;
+    ga.zero_counter = (fast && l == 0) ? fb_count : nullptr;
     profile_begin(s);
-    const cudaError_t ge = launch_gemm(epi, p.G, s, tmA, tmB, ga);
+    const cudaError_t ge = launch_gemm(epi, p.pair, p.G, s, (x_is_operand && l == 0) ? tmX : tmA, tmB, ga);
     profile_end(s);
     note_launch();
     if (ge != cudaSuccess) return RVQ_ERR_CUDA;
@@ -1078,6 +1524,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ra.Tc = p.Tc;
     ra.G = p.G;
     ra.maxs = p.maxs;
+    ra.pair = p.pair ? 1 : 0;
     ra.U = p.U;
     ra.cand = cand;
     ra.rowstat = rowstat;
@@ -1090,8 +1537,23 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ra.fb_count = fb_count + l;
     ra.status = status;
     ra.last = l == L - 1;
-    cudaError_t e1, e2;
-    if (cb_dtype == RVQ_BF16) {
+    ra.src = l == 0 && fast ? features : static_cast<const void *>(R);
+    ra.fb_next = (fast && l + 1 < L) ? fb_count + l + 1 : nullptr;
+    ra.offsets = (fast && l == 0) ? offsets : nullptr;
+    ra.B = B;
+    cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+    if (fast) {
+      const unsigned rb = static_cast<unsigned>(row_blocks);
+      if (l > 0)
+        e1 = cb_dtype == RVQ_BF16 ? launch_rows_fast<true, SRC_R>(ra, nch, rb, fb_blocks, fb_smem, s)
+                                  : launch_rows_fast<false, SRC_R>(ra, nch, rb, fb_blocks, fb_smem, s);
+      else if (f_dtype == RVQ_BF16)
+        e1 = cb_dtype == RVQ_BF16 ? launch_rows_fast<true, SRC_X_BF16>(ra, nch, rb, fb_blocks, fb_smem, s)
+                                  : launch_rows_fast<false, SRC_X_BF16>(ra, nch, rb, fb_blocks, fb_smem, s);
+      else
+        e1 = cb_dtype == RVQ_BF16 ? launch_rows_fast<true, SRC_X_F32>(ra, nch, rb, fb_blocks, fb_smem, s)
+                                  : launch_rows_fast<false, SRC_X_F32>(ra, nch, rb, fb_blocks, fb_smem, s);
+    } else if (cb_dtype == RVQ_BF16) {
       e1 = launch_pdl(rescore_kernel<true>, dim3(static_cast<unsigned>(row_blocks)), dim3(256), 0, s, ra);
       e2 = launch_pdl(fallback_kernel<true>, dim3(fb_blocks), dim3(256), fb_smem, s, ra);
     } else {
