@@ -15,7 +15,11 @@
 namespace rvq {
 
 constexpr int kDecodeWarps = 8;
-constexpr int kDecodeLevelGroup = 8;  // gathers issued together before they are summed
+constexpr int kDecodeLevelGroup = 8;  // gathers of one row issued together before they are summed
+#ifndef RVQ_DECODE_ROWS
+#define RVQ_DECODE_ROWS 1
+#endif
+constexpr int kDecodeRows = RVQ_DECODE_ROWS;  // rows per warp: their gathers are in flight together
 
 // VEC consecutive elements of one codeword row, widened to fp32.
 template <bool CB_BF16, int VEC>
@@ -72,15 +76,80 @@ struct Gather<false, 4> {  // 16-byte load of 4 fp32
   }
 };
 
-// One warp per row and slice of 32*VEC columns; lane = VEC consecutive columns.  The gathers of
-// eight levels are issued back to back with no branch between them (an out-of-range id or a
-// lane past D reads a clamped, valid address and is masked afterwards), then summed in
-// ascending level order.
-template <bool CB_BF16, int VEC>
+// One warp per R rows and a slice of 32*VEC columns; lane = VEC consecutive columns.  The gathers of
+// eight levels of all R rows are issued back to back with no branch between them (an out-of-range
+// id or a lane past D reads a clamped, valid address and is masked afterwards), then each row is
+// summed in ascending level order.
+template <bool CB_BF16, int VEC, int R>
 __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t *__restrict__ ids, int64_t N,
                                                                   int L, const void *__restrict__ cb, int K,
                                                                   int D, float *__restrict__ recon,
                                                                   int32_t *status) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t n0 = (static_cast<int64_t>(blockIdx.x) * kDecodeWarps + (threadIdx.x >> 5)) * R;
+  if (n0 >= N) return;  // whole warp
+  const int col = blockIdx.y * (32 * VEC) + lane * VEC;
+  const bool active = col < D;
+  const int colc = active ? col : 0;
+  int id_lo[R], id_hi[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t n = n0 + r < N ? n0 + r : N - 1;  // rows past N repeat the last row, never stored
+    id_lo[r] = lane < L ? __ldg(ids + n * L + lane) : 0;
+    id_hi[r] = lane + 32 < L ? __ldg(ids + n * L + 32 + lane) : 0;
+  }
+  float acc[R][VEC];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) acc[r][k] = 0.f;
+  bool bad = false;
+  for (int l0 = 0; l0 < L; l0 += kDecodeLevelGroup) {
+    Gather<CB_BF16, VEC> g[R][kDecodeLevelGroup];
+    bool use[R][kDecodeLevelGroup];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int src = l0 < 32 ? id_lo[r] : id_hi[r];
+#pragma unroll
+      for (int j = 0; j < kDecodeLevelGroup; ++j) {
+        const int l = l0 + j;
+        const int id = __shfl_sync(0xffffffffu, src, l & 31);
+        const bool lv = l < L;
+        const bool ok = lv && static_cast<unsigned>(id) < static_cast<unsigned>(K);
+        bad |= lv && !ok && n0 + r < N;
+        use[r][j] = ok;
+        const int lc = lv ? l : L - 1;
+        g[r][j].load(cb, (static_cast<int64_t>(lc) * K + (ok ? id : 0)) * D + colc);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < kDecodeLevelGroup; ++j)
+        if (use[r][j]) g[r][j].add_to(acc[r]);
+  }
+  if (active) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (n0 + r >= N) break;
+      float4 *dst = reinterpret_cast<float4 *>(recon + (n0 + r) * D + col);
+#pragma unroll
+      for (int k = 0; k < VEC; k += 4)
+        __stcs(dst + k / 4, make_float4(acc[r][k], acc[r][k + 1], acc[r][k + 2], acc[r][k + 3]));
+    }
+  }
+  if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
+}
+
+// The same with the number of levels known at compile time (LC <= 16): one row per warp, all LC
+// gathers in flight at once, few registers, so many warps per SM keep the L2 busy.
+template <bool CB_BF16, int VEC, int LC>
+__global__ void __launch_bounds__(kDecodeWarps * 32, 6) decode_fixed_kernel(const int32_t *__restrict__ ids,
+                                                                           int64_t N, const void *__restrict__ cb,
+                                                                           int K, int D, float *__restrict__ recon,
+                                                                           int32_t *status) {
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
@@ -89,32 +158,24 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t
   const int col = blockIdx.y * (32 * VEC) + lane * VEC;
   const bool active = col < D;
   const int colc = active ? col : 0;
-  const int32_t *row_ids = ids + n * L;
-  const int id_lo = lane < L ? __ldg(row_ids + lane) : 0;
-  const int id_hi = lane + 32 < L ? __ldg(row_ids + 32 + lane) : 0;
+  const int myid = lane < LC ? __ldg(ids + n * LC + lane) : 0;
+  Gather<CB_BF16, VEC> g[LC];
+  bool use[LC];
+  bool bad = false;
+#pragma unroll
+  for (int l = 0; l < LC; ++l) {
+    const int id = __shfl_sync(0xffffffffu, myid, l);
+    const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(K);
+    bad |= !ok;
+    use[l] = ok;
+    g[l].load(cb, (static_cast<int64_t>(l) * K + (ok ? id : 0)) * D + colc);
+  }
   float acc[VEC];
 #pragma unroll
   for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-  bool bad = false;
-  for (int l0 = 0; l0 < L; l0 += kDecodeLevelGroup) {
-    Gather<CB_BF16, VEC> g[kDecodeLevelGroup];
-    bool use[kDecodeLevelGroup];
-    const int src = l0 < 32 ? id_lo : id_hi;
 #pragma unroll
-    for (int j = 0; j < kDecodeLevelGroup; ++j) {
-      const int l = l0 + j;
-      const int id = __shfl_sync(0xffffffffu, src, l & 31);
-      const bool lv = l < L;
-      const bool ok = lv && static_cast<unsigned>(id) < static_cast<unsigned>(K);
-      bad |= lv && !ok;
-      use[j] = ok;
-      const int lc = lv ? l : L - 1;
-      g[j].load(cb, (static_cast<int64_t>(lc) * K + (ok ? id : 0)) * D + colc);
-    }
-#pragma unroll
-    for (int j = 0; j < kDecodeLevelGroup; ++j)
-      if (use[j]) g[j].add_to(acc);
-  }
+  for (int l = 0; l < LC; ++l)
+    if (use[l]) g[l].add_to(acc);
   if (active) {
     float4 *dst = reinterpret_cast<float4 *>(recon + n * D + col);
 #pragma unroll
@@ -123,18 +184,50 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t
   if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
 }
 
+template <bool CB_BF16, int VEC, int LC>
+cudaError_t launch_fixed(const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon, int32_t *status,
+                         cudaStream_t s) {
+  const int64_t gx = (N + kDecodeWarps - 1) / kDecodeWarps;
+  const int gy = (D + 32 * VEC - 1) / (32 * VEC);
+  if (gx > 0x7FFFFFFFLL || gy > 65535) return cudaErrorInvalidValue;
+  return launch_pdl(decode_fixed_kernel<CB_BF16, VEC, LC>, dim3(static_cast<unsigned>(gx), gy),
+                    dim3(kDecodeWarps * 32), 0, s, ids, N, cb, K, D, recon, status);
+}
+
+template <bool CB_BF16, int VEC, int LC = 1>
+cudaError_t dispatch_fixed(int L, const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon,
+                           int32_t *status, cudaStream_t s) {
+  if constexpr (LC > 16) {
+    return cudaErrorInvalidValue;
+  } else {
+    if (L == LC) return launch_fixed<CB_BF16, VEC, LC>(ids, N, cb, K, D, recon, status, s);
+    return dispatch_fixed<CB_BF16, VEC, LC + 1>(L, ids, N, cb, K, D, recon, status, s);
+  }
+}
+
 template <bool CB_BF16, int VEC>
 cudaError_t launch_decode_t(const int32_t *ids, int64_t N, int L, const void *cb, int K, int D, float *recon,
                             int32_t *status, cudaStream_t s, dim3 grid) {
-  return launch_pdl(decode_kernel<CB_BF16, VEC>, grid, dim3(kDecodeWarps * 32), 0, s, ids, N, L, cb, K, D, recon,
-                    status);
+  return launch_pdl(decode_kernel<CB_BF16, VEC, kDecodeRows>, grid, dim3(kDecodeWarps * 32), 0, s, ids, N, L, cb, K,
+                    D, recon, status);
 }
 
 int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_dtype, int K, int D, float *recon,
                   int32_t *status, cudaStream_t s) {
   if (N == 0) return RVQ_OK;
+  if (L <= 16) {
+    cudaError_t e;
+    if (cb_dtype == RVQ_BF16)
+      e = D % 8 == 0 ? dispatch_fixed<true, 8>(L, ids, N, cb, K, D, recon, status, s)
+                     : dispatch_fixed<true, 4>(L, ids, N, cb, K, D, recon, status, s);
+    else
+      e = dispatch_fixed<false, 4>(L, ids, N, cb, K, D, recon, status, s);
+    note_launch();
+    return e == cudaSuccess ? RVQ_OK : e == cudaErrorInvalidValue ? RVQ_ERR_UNSUPPORTED : RVQ_ERR_CUDA;
+  }
   const int vec = (cb_dtype == RVQ_BF16 && D % 8 == 0) ? 8 : 4;
-  const int64_t gx = (N + kDecodeWarps - 1) / kDecodeWarps;
+  const int64_t rows_per_block = static_cast<int64_t>(kDecodeWarps) * kDecodeRows;
+  const int64_t gx = (N + rows_per_block - 1) / rows_per_block;
   const int gy = (D + 32 * vec - 1) / (32 * vec);
   if (gx > 0x7FFFFFFFLL || gy > 65535) return RVQ_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
