@@ -333,41 +333,73 @@ def run_ours(args, rank, world, local_rank):
     decode_gbs = decode_bytes / (breakdown["decode"] / 1e3) / 1e9
 
     # -------------------------------------------------- end to end through host buffers
+    # Every step copies its features from pinned host memory and its ids + decoded recon back.
+    # Two buffer sets and separate copy/compute streams let step k's copies overlap the compute of
+    # its neighbours, as a pipeline tokenizing a stream of images would run.
     e2e = None
     if not args.no_e2e:
+        copy_in = torch.cuda.Stream(dev)
+        copy_out = torch.cuda.Stream(dev)
         if detok_only:
-            h_in = torch.from_numpy(g["planted"]).pin_memory()
-            d_in = torch.empty_like(ids)
+            h_in = [torch.from_numpy(g["planted"]).pin_memory() for _ in range(2)]
+            d_in = [torch.empty_like(ids) for _ in range(2)]
         else:
-            h_in = (torch.from_numpy(g["x"]).to(torch.bfloat16) if spec.f_dtype == "bf16"
-                    else torch.from_numpy(g["x"])).pin_memory()
-            d_in = torch.empty_like(x)
-        h_ids = torch.empty((N, L), dtype=torch.int32).pin_memory()
-        h_rec = torch.empty((N, D), dtype=torch.float32).pin_memory()
-        e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        for k in range(args.steps + 2):
-            flush.zero_()
-            kk = k - 2
-            if kk >= 0:
-                e_starts[kk].record(stream)
-            d_in.copy_(h_in, non_blocking=True)
+            src = torch.from_numpy(g["x"]).to(torch.bfloat16) if spec.f_dtype == "bf16" else torch.from_numpy(g["x"])
+            h_in = [src.pin_memory() for _ in range(2)]
+            d_in = [torch.empty_like(x) for _ in range(2)]
+        d_ids = [torch.empty_like(ids) for _ in range(2)]
+        d_rec = [torch.empty_like(rec2) for _ in range(2)]
+        d_x = [torch.empty_like(x) for _ in range(2)] if detok_only else None
+        h_ids = [torch.empty((N, L), dtype=torch.int32).pin_memory() for _ in range(2)]
+        h_rec = [torch.empty((N, D), dtype=torch.float32).pin_memory() for _ in range(2)]
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def pipe_step(k):
+            b = k % 2
+            with torch.cuda.stream(copy_in):
+                if k >= 2:
+                    copy_in.wait_event(ev_done[b])       # the compute of step k-2 is done with d_in[b]
+                d_in[b].copy_(h_in[b], non_blocking=True)
+                ev_in[b].record(copy_in)
+            stream.wait_event(ev_in[b])
+            if k >= 2:
+                stream.wait_event(ev_out[b])             # step k-2's results have left d_ids/d_rec[b]
             if detok_only:
-                xin = tok.decode(d_in, out=x, check=False)
-                step(xin)
+                xin = tok.decode(d_in[b], out=d_x[b], check=False)
             else:
-                step(d_in)
-            h_ids.copy_(ids, non_blocking=True)
-            h_rec.copy_(rec2, non_blocking=True)
-            if kk >= 0:
-                e_ends[kk].record(stream)
+                xin = d_in[b]
+            check(mvt.rvq_build_norms(cb, tok.cb_dtype, L, K, D, tok.norms, tok.level_stats, tok.operand, stream),
+                  "rvq_build_norms")
+            check(mvt.rvq_encode(xin, f_code, N, D, cb, tok.cb_dtype, tok.operand, tok.norms, tok.level_stats, L,
+                                 K, off, B, d_ids[b], res, None, fb, ws, ws_bytes, status, stream), "rvq_encode")
+            check(mvt.rvq_decode(d_ids[b], N, L, cb, tok.cb_dtype, K, D, d_rec[b], status, stream), "rvq_decode")
+            ev_done[b].record(stream)
+            with torch.cuda.stream(copy_out):
+                copy_out.wait_event(ev_done[b])
+                h_ids[b].copy_(d_ids[b], non_blocking=True)
+                h_rec[b].copy_(d_rec[b], non_blocking=True)
+                ev_out[b].record(copy_out)
+
+        for k in range(2):
+            pipe_step(k)
         torch.cuda.synchronize(dev)
-        e_ms = sharding.max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), dev)
-        h2d = h_in.numel() * h_in.element_size()
-        d2h = h_ids.numel() * 4 + h_rec.numel() * 4
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(copy_in)
+        for k in range(args.steps):
+            pipe_step(k)
+        copy_out.wait_event(ev_out[(args.steps - 1) % 2])
+        t1.record(copy_out)
+        torch.cuda.synchronize(dev)
+        e_ms = sharding.max_over_ranks(t0.elapsed_time(t1), dev)
+        h2d = h_in[0].numel() * h_in[0].element_size()
+        d2h = h_ids[0].numel() * 4 + h_rec[0].numel() * 4
         e2e = {"value": N * world / (e_ms / args.steps / 1e3) / 1e6, "unit": "Mtokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e_ms / args.steps}
+               "ms_per_step": e_ms / args.steps,
+               "pipeline": "2 buffer sets; copy-in, compute and copy-out streams overlap across steps"}
 
     # -------------------------------------------------- roofline of the distance GEMM
     long_step = ms_per_step > 20.0

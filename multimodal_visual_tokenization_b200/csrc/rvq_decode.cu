@@ -20,6 +20,10 @@ constexpr int kDecodeLevelGroup = 8;  // gathers of one row issued together befo
 #define RVQ_DECODE_ROWS 1
 #endif
 constexpr int kDecodeRows = RVQ_DECODE_ROWS;  // rows per warp: their gathers are in flight together
+#ifndef RVQ_DECODE_BF16_VEC
+#define RVQ_DECODE_BF16_VEC 8
+#endif
+constexpr int kBf16Vec = RVQ_DECODE_BF16_VEC;  // bf16 elements per lane per gather (8: 256-column slices)
 
 // VEC consecutive elements of one codeword row, widened to fp32.
 template <bool CB_BF16, int VEC>
@@ -218,8 +222,8 @@ int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_d
   if (L <= 16) {
     cudaError_t e;
     if (cb_dtype == RVQ_BF16)
-      e = D % 8 == 0 ? dispatch_fixed<true, 8>(L, ids, N, cb, K, D, recon, status, s)
-                     : dispatch_fixed<true, 4>(L, ids, N, cb, K, D, recon, status, s);
+      e = (D % 8 == 0 && kBf16Vec == 8) ? dispatch_fixed<true, 8>(L, ids, N, cb, K, D, recon, status, s)
+                                        : dispatch_fixed<true, 4>(L, ids, N, cb, K, D, recon, status, s);
     else
       e = dispatch_fixed<false, 4>(L, ids, N, cb, K, D, recon, status, s);
     note_launch();

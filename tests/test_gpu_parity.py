@@ -240,3 +240,54 @@ def test_launch_count_and_profile_hooks():
     mvt.rvq_profile_enable(False)
     assert code == 0 and n == g["spec"].L and ms > 0
     assert mvt.rvq_launch_count() - before == 1 + 3 * g["spec"].L
+
+
+def test_wide_features_use_streaming_rows():
+    """D > 1024 takes the path that materialises the fp32 residual and streams rows."""
+    rng = np.random.Generator(np.random.PCG64(27))
+    L, K, D, N = 3, 300, 2048, 200
+    C = rng.standard_normal((L, K, D)).astype(np.float32) * (0.5 ** np.arange(L, dtype=np.float32))[:, None, None]
+    x = workloads.round_bf16(C[0][rng.integers(0, K, N)] + 0.1 * rng.standard_normal((N, D)).astype(np.float32))
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    full_check(x, C, ids, res, rec)
+
+
+def test_fewer_codewords_than_list_entries():
+    rng = np.random.Generator(np.random.PCG64(28))
+    for K in (1, 3, 7):
+        C = rng.standard_normal((2, K, 64)).astype(np.float32)
+        x = rng.standard_normal((150, 64)).astype(np.float32)
+        _, ids, res, rec, fb = run_encode(x, C)
+        full_check(x, C, ids, res, rec)
+
+
+def test_decode_many_levels_generic_path():
+    """More than 16 levels uses the runtime-level decode kernel."""
+    rng = np.random.Generator(np.random.PCG64(29))
+    L, K, D, N = 20, 37, 96, 333
+    C = workloads.round_bf16(rng.standard_normal((L, K, D)).astype(np.float32))
+    ids = rng.integers(0, K, size=(N, L)).astype(np.int32)
+    for dt in ("f32", "bf16"):
+        tok = mvt.Tokenizer(dev(C, dt))
+        rec = tok.decode(torch.from_numpy(ids).cuda())
+        torch.cuda.synchronize()
+        parity.check_recon(None, C, np.arange(N), ids, recon_gpu=rec.cpu().numpy())
+
+
+def test_cta_pair_kernel_matches_oracle():
+    """The optional 2-CTA (cta_group::2) distance GEMM, selected by RVQ_PAIR=1 in a fresh process."""
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, torch, workloads\n"
+        "from tests import parity, test_gpu_parity as t\n"
+        "g = workloads.generate('image', n_override=700)\n"
+        "_, ids, res, rec, fb = t.run_encode(g['x'], g['codebooks'], 'bf16', 'f32')\n"
+        "t.full_check(g['x'], g['codebooks'], ids, res, rec)\n"
+        "print('pair ok')\n")
+    import os
+    env = dict(os.environ, RVQ_PAIR="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0 and "pair ok" in out.stdout, out.stdout[-2000:] + out.stderr[-2000:]
