@@ -165,8 +165,10 @@ RVQ_API const char *rvq_status_str(int status);
  * rvq_launch_count: number of kernels this library has launched since it was loaded.
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on
  *   its stream (not for use inside stream capture); rvq_profile_enable(0) stops and clears.
- * rvq_profile_read: synchronises on the recorded events and returns the number of distance-
- *   GEMM launches and their summed device time in milliseconds since the last enable.
+ * rvq_profile_read: synchronises on the recorded events and returns the number of RVQ levels the
+ *   bracketed launches covered (a per-level distance-GEMM launch counts 1; the all-levels persistent
+ *   encode kernel, which also runs the certificate phases, counts L) and their summed device time
+ *   in milliseconds since the last enable.
  */
 RVQ_API int64_t rvq_launch_count(void);
 RVQ_API int rvq_profile_enable(int enable);

@@ -24,6 +24,7 @@ struct Profiler {
   std::mutex mu;
   bool on = false;
   std::vector<cudaEvent_t> pool;  // even = start, odd = end
+  std::vector<int> levels;        // RVQ levels covered by each bracketed launch
   size_t used = 0;                // events handed out since enable
 };
 Profiler &prof() {
@@ -52,13 +53,17 @@ void profile_begin(cudaStream_t s) {
   if (e) cudaEventRecord(e, s);
 }
 
-void profile_end(cudaStream_t s) {
+void profile_end(cudaStream_t s, int levels) {
   Profiler &p = prof();
   std::lock_guard<std::mutex> g(p.mu);
   if (!p.on) return;
   if (p.used % 2 != 1) return;
   cudaEvent_t e = take_event();
-  if (e) cudaEventRecord(e, s);
+  if (e) {
+    cudaEventRecord(e, s);
+    p.levels.resize(p.used / 2);
+    p.levels.back() = levels;
+  }
 }
 
 }  // namespace rvq
@@ -85,6 +90,7 @@ int rvq_profile_enable(int enable) {
   std::lock_guard<std::mutex> g(p.mu);
   p.on = enable != 0;
   p.used = 0;
+  p.levels.clear();
   return RVQ_OK;
 }
 
@@ -99,7 +105,7 @@ int rvq_profile_read(int64_t *gemm_launches, double *gemm_ms) {
     float ms = 0.f;
     if (cudaEventElapsedTime(&ms, p.pool[i], p.pool[i + 1]) != cudaSuccess) return RVQ_ERR_CUDA;
     total += ms;
-    ++n;
+    n += i / 2 < p.levels.size() ? p.levels[i / 2] : 1;
   }
   *gemm_launches = n;
   *gemm_ms = total;

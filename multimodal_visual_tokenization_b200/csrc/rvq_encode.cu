@@ -57,7 +57,8 @@ constexpr int BN = 256;       // codewords per tile (UMMA N)
 constexpr int BK = 64;        // bf16 elements per k-block = one 128-byte swizzle row
 constexpr int UK = 16;        // K of one kind::f16 UMMA
 constexpr int TOPK = 8;
-constexpr int MAX_SLOTS = 8;  // partial lists per row tile (bounds the rescore merge)
+constexpr int MAX_SLOTS = 16;  // partial lists per row tile (bounds the rescore merge)
+constexpr int CPL = MAX_SLOTS * TOPK / 32;  // candidates per lane when one warp merges a row's lists
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int TMEM_COLS = 2 * BN;
 // Norm term of the distance, folded into the GEMM as one extra K=16 step: A_aug rows are
@@ -98,7 +99,8 @@ struct GemmCfg {
   static constexpr int AUG_B_OFF = AUG_A_OFF + AUG_A_BYTES;                // 2 slots
   static constexpr int MERGE_OFF = AUG_B_OFF + 2 * AUG_B_BYTES;            // (GROUPS-1) x 128 x 8 x 8 B
   static constexpr int BAR_OFF = MERGE_OFF + (GROUPS - 1) * BM * TOPK * 8;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;                        // + barriers + alignment slack
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;                        // + barriers + alignment slack
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB per-block limit");
 };
 
 struct GemmArgs {
@@ -178,6 +180,36 @@ __device__ __forceinline__ void cx_idx(float &a, float &b, int &ia, int &ib) {
   ib = sw ? tia : ib;
 }
 // Merge the chunk of 32 keys d[] (columns c0 + j, all finite) into the running list.
+// d[j] for a run-time j in [0, 32) as a tree of selects (no local-memory copy of d).
+__device__ __forceinline__ float pick32(const float (&d)[32], int j) {
+  float t16[16], t8[8], t4[4], t2[2];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t16[i] = (j & 1) ? d[2 * i + 1] : d[2 * i];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t8[i] = (j & 2) ? t16[2 * i + 1] : t16[2 * i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) t4[i] = (j & 4) ? t8[2 * i + 1] : t8[2 * i];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) t2[i] = (j & 8) ? t4[2 * i + 1] : t4[2 * i];
+  return (j & 16) ? t2[1] : t2[0];
+}
+
+// Insert the chunk entries below the current 8th best, in column order (the same result as
+// offering all 32 to topk_insert in order).  The entries are found from a bit mask and fetched
+// with pick32, so the loop runs as often as the busiest lane has entries and stays small in code.
+__device__ __forceinline__ void topk_insert_few(float (&bd)[TOPK], int (&bi)[TOPK], const float (&d)[32], int c0) {
+  const float thr = bd[TOPK - 1];
+  unsigned mask = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) mask |= (d[j] < thr ? 1u : 0u) << j;
+#pragma unroll 1
+  while (__any_sync(0xffffffffu, mask != 0)) {
+    const int j = __ffs(mask) - 1;
+    mask &= mask - 1;
+    if (j >= 0) topk_insert(bd, bi, pick32(d, j), c0 + j);
+  }
+}
+
 __device__ __forceinline__ void topk_merge_chunk(float (&bd)[TOPK], int (&bi)[TOPK], const float (&d)[32], int c0) {
   float k[32];
 #pragma unroll
@@ -495,13 +527,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
           mbar_arrive(mready);
         } else {
           if (!mbar_wait(mready, nflush & 1u, abort_flag)) return false;
-          for (int gg = 1; gg < C::GROUPS; ++gg) {
-            const float2 *other = mbuf + (static_cast<int64_t>(gg - 1) * BM + row_in_tile) * TOPK;
-#pragma unroll
-            for (int t = 0; t < TOPK; ++t) {
-              const float2 e = other[t];
-              if (e.x < bd[TOPK - 1]) topk_insert(bd, bi, e.x, __float_as_int(e.y));
-            }
+          #pragma unroll 1
+          for (int e8 = 0; e8 < (C::GROUPS - 1) * TOPK; ++e8) {
+            const float2 e = mbuf[(static_cast<int64_t>(e8 / TOPK) * BM + row_in_tile) * TOPK + e8 % TOPK];
+            if (e.x < bd[TOPK - 1]) topk_insert(bd, bi, e.x, __float_as_int(e.y));
           }
           mbar_arrive(mdone);
         }
@@ -588,10 +617,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
         if (__popc(need) >= kMergeLanes) {
           topk_merge_chunk(bd, bi, d, c0);  // many lanes: one branch-free merge for the warp
         } else if (need) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (__any_sync(0xffffffffu, d[j] < bd[TOPK - 1])) topk_insert(bd, bi, d[j], c0 + j);
-          }
+          topk_insert_few(bd, bi, d, c0);
         }
       }
     }
@@ -717,6 +743,8 @@ struct RowArgs {
   int Tc, G, maxs;
   int pair;  // units span 256 rows (CTA pairs) instead of 128
   int64_t U;
+  int64_t rt0;  // first row tile of the unit range, else 0
+  int nslots;   // > 0: every row tile has exactly nslots candidate lists (all-levels kernel)
   const float2 *cand;
   float2 *rowstat;
   float *R;
@@ -747,8 +775,8 @@ __device__ __forceinline__ float4 ld_src4(const void *p, int64_t off) {
     return make_float4(x.x, x.y, y.x, y.y);
   } else if constexpr (SRC == SRC_X_F32) {
     return __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off));
-  } else {  // the running residual, written by the previous level: no read-only cache
-    return *reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off);
+  } else {  // the running residual, written by the previous level: read at L2, never a stale L1 line
+    return __ldcg(reinterpret_cast<const float4 *>(static_cast<const float *>(p) + off));
   }
 }
 
@@ -810,34 +838,35 @@ __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
   if (n >= a.N) return;
   const int64_t rt = n / BM;
   const int rin = static_cast<int>(n - rt * BM);
-  const int64_t ut = a.pair ? (rt >> 1) : rt;  // the unit row tile this 128-row tile belongs to
+  const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;  // the unit row tile this 128-row tile belongs to
   const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
   const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
   const int ncand = (c1 - c0 + 1) * TOPK;
 
-  float dv[2];
-  int iv[2];
+  float dv[CPL];
+  int iv[CPL];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < CPL; ++h) {
     const int e = lane + 32 * h;
     dv[h] = inf_f();
     iv[h] = -1;
     if (e < ncand) {
       const int slot = e / TOPK, t = e - slot * TOPK;
-      const float2 c = a.cand[((rt * a.maxs + slot) * BM + rin) * TOPK + t];
+      const float2 c = __ldcg(a.cand + ((rt * a.maxs + slot) * BM + rin) * TOPK + t);
       dv[h] = c.x;
       iv[h] = __float_as_int(c.y);
     }
   }
   // T: smallest score that some list dropped (a list's last entry; +inf if the list is short)
-  float tl = inf_f();
+  float tl = inf_f(), ml = inf_f();
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < CPL; ++h) {
     const int e = lane + 32 * h;
     if (e < ncand && (e % TOPK) == TOPK - 1) tl = fminf(tl, dv[h]);
+    ml = fminf(ml, dv[h]);
   }
   const float T = warp_min_f(tl);
-  const float dmin = warp_min_f(fminf(dv[0], dv[1]));
+  const float dmin = warp_min_f(ml);
   // + the index bits the chunk-merge path stores in candidate keys (relative change < 2^-18)
   const float E = error_bound(a.stats, a.rowstat[n], a.D) +
                   7.62939453125e-06f * (fabsf(dmin) + (T < 1e30f ? fabsf(T) : 0.f));  // 2^-17
@@ -855,7 +884,7 @@ __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
   int best_id = 0x7fffffff;
   const float lim = dmin + 2.f * E;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < CPL; ++h) {
     unsigned mask = __ballot_sync(0xffffffffu, iv[h] >= 0 && dv[h] <= lim);
     while (mask) {
       const int src = __ffs(mask) - 1;
@@ -952,27 +981,58 @@ __global__ void __launch_bounds__(256) fallback_kernel(const RowArgs a) {
 // the candidate lists, the row and the winner's codeword are each read once, and the updated
 // residual, its bf16 operand copy and row statistics are written from registers.
 
-template <bool CB_BF16, int SRC, int NCH>
-__global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
-  griddep_launch_dependents();
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (gtid == 0 && a.fb_next) *a.fb_next = 0;
-  if (a.offsets) {  // packed-batch bookkeeping: offsets[0] = 0, non-decreasing, offsets[B] = N
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t b = gtid; b < a.B; b += nthreads)
-      if (a.offsets[b] > a.offsets[b + 1]) set_status(a.status, RVQ_ERR_ARG);
-    if (gtid == 0 && (a.offsets[0] != 0 || a.offsets[a.B] != a.N)) set_status(a.status, RVQ_ERR_ARG);
+// Packed-batch bookkeeping: offsets[0] = 0, non-decreasing, offsets[B] = N (checked, not used).
+__device__ __forceinline__ void check_offsets(const RowArgs &a, int64_t gtid, int64_t nthreads) {
+  for (int64_t b = gtid; b < a.B; b += nthreads)
+    if (a.offsets[b] > a.offsets[b + 1]) set_status(a.status, RVQ_ERR_ARG);
+  if (gtid == 0 && (a.offsets[0] != 0 || a.offsets[a.B] != a.N)) set_status(a.status, RVQ_ERR_ARG);
+}
+
+// r -= c for a register-resident row (element lane*4 + 128k of chunk k), then the ids entry and,
+// unless this was the last level, the next level's bf16 operand row and its rounding statistics.
+template <int NCH>
+__device__ __forceinline__ void apply_row(const RowArgs &a, int64_t n, const float4 (&rv)[NCH],
+                                          const float4 (&c)[NCH], int id, int lane) {
+  float e2 = 0.f, q2 = 0.f;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    if (i >= a.D) break;
+    float4 v = rv[k];
+    v.x -= c[k].x;
+    v.y -= c[k].y;
+    v.z -= c[k].z;
+    v.w -= c[k].w;
+    *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
+    if (!a.last) {
+      float4 q;
+      store_bf16x4(a.Rt + n * a.D + i, v, &q);
+      const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+      e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+      q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+    }
   }
-  const int64_t n = gtid >> 5;
-  if (n >= a.N) return;
+  if (!a.last) {
+    e2 = warp_sum_f(e2);
+    q2 = warp_sum_f(q2);
+    if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
+  }
+  if (lane == 0) a.ids[n * a.L + a.l] = id;
+}
+
+// Certificate, exact rescore when needed, and the residual update of row n (one warp).  Returns
+// whether the row was settled; an uncertified row is appended to a.fb_list when that is set.
+template <bool CB_BF16, int SRC, int NCH>
+__device__ __forceinline__ bool rescore_row(const RowArgs &a, int64_t n, int lane) {
   const int64_t rt = n / BM;
   const int rin = static_cast<int>(n - rt * BM);
-  const int64_t ut = a.pair ? (rt >> 1) : rt;
-  const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
-  const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
-  const int ncand = (c1 - c0 + 1) * TOPK;
+  int ncand = a.nslots * TOPK;
+  if (a.nslots <= 0) {
+    const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;
+    const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
+    const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
+    ncand = (c1 - c0 + 1) * TOPK;
+  }
 
   // independent loads first: the residual row and the candidate lists
   float4 rv[NCH];
@@ -981,22 +1041,22 @@ __global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
     const int i = lane * 4 + k * 128;
     rv[k] = i < a.D ? ld_src4<SRC>(a.src, n * a.D + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  float dv[2];
-  int iv[2];
+  float dv[CPL];
+  int iv[CPL];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < CPL; ++h) {
     const int e = lane + 32 * h;
     dv[h] = inf_f();
     iv[h] = -1;
     if (e < ncand) {
       const int slot = e / TOPK, t = e - slot * TOPK;
-      const float2 c = a.cand[((rt * a.maxs + slot) * BM + rin) * TOPK + t];
+      const float2 c = __ldcg(a.cand + ((rt * a.maxs + slot) * BM + rin) * TOPK + t);
       dv[h] = c.x;
       iv[h] = __float_as_int(c.y);
     }
   }
   float2 rs = make_float2(0.f, 0.f);
-  if constexpr (SRC != SRC_X_BF16) rs = a.rowstat[n];
+  if constexpr (SRC != SRC_X_BF16) rs = __ldcg(a.rowstat + n);
 
   // r is its own bf16 copy when it comes straight from bf16 features: e_r = 0, ||r~|| = ||r||
   if constexpr (SRC == SRC_X_BF16) {
@@ -1006,25 +1066,33 @@ __global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
     rs = make_float2(0.f, __fsqrt_ru(1.0001f * warp_sum_f(q)));
   }
 
-  float tl = inf_f();
+  float tl = inf_f(), ml = inf_f();
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < CPL; ++h) {
     const int e = lane + 32 * h;
     if (e < ncand && (e % TOPK) == TOPK - 1) tl = fminf(tl, dv[h]);
+    ml = fminf(ml, dv[h]);
   }
   const float T = warp_min_f(tl);
-  const float dmin = warp_min_f(fminf(dv[0], dv[1]));
+  const float dmin = warp_min_f(ml);
   const float E = error_bound(a.stats, rs, a.D) + 7.62939453125e-06f * (fabsf(dmin) + (T < 1e30f ? fabsf(T) : 0.f));
   const float lim = dmin + 2.f * E;
-  const unsigned pm0 = __ballot_sync(0xffffffffu, iv[0] >= 0 && dv[0] <= lim);
-  const unsigned pm1 = __ballot_sync(0xffffffffu, iv[1] >= 0 && dv[1] <= lim);
+  unsigned pm[CPL];
+  int nplaus = 0;
+#pragma unroll
+  for (int h = 0; h < CPL; ++h) {
+    pm[h] = __ballot_sync(0xffffffffu, iv[h] >= 0 && dv[h] <= lim);
+    nplaus += __popc(pm[h]);
+  }
 
   int best_id = 0x7fffffff;
   float4 cbest[NCH];
-  if (__popc(pm0) + __popc(pm1) == 1 && T - dmin > 2.f * E) {
+  if (nplaus == 1 && T - dmin > 2.f * E) {
     // One candidate within 2E of the best score and every dropped score more than 2E above it:
     // its true distance is below every other codeword's, so no exact rescore is needed.
-    best_id = pm0 ? __shfl_sync(0xffffffffu, iv[0], __ffs(pm0) - 1) : __shfl_sync(0xffffffffu, iv[1], __ffs(pm1) - 1);
+#pragma unroll
+    for (int h = 0; h < CPL; ++h)
+      if (pm[h]) best_id = __shfl_sync(0xffffffffu, iv[h], __ffs(pm[h]) - 1);
     const int64_t coff = (static_cast<int64_t>(a.l) * a.K + best_id) * a.D;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
@@ -1040,10 +1108,8 @@ __global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
     rr = warp_sum_d(rr);
     double best = inf_d();
 #pragma unroll
-    for (int k = 0; k < NCH; ++k) cbest[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      unsigned mask = h == 0 ? pm0 : pm1;
+    for (int h = 0; h < CPL; ++h) {
+      unsigned mask = pm[h];
       while (mask) {
         const int srcl = __ffs(mask) - 1;
         mask &= mask - 1;
@@ -1066,46 +1132,121 @@ __global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
         if (dd < best || (dd == best && id < best_id)) {
           best = dd;
           best_id = id;
-#pragma unroll
-          for (int k = 0; k < NCH; ++k) cbest[k] = c[k];
         }
       }
     }
     const bool certified =
         best_id != 0x7fffffff && (best - rr) < (static_cast<double>(T) - static_cast<double>(E));
     if (!certified) {
-      if (lane == 0) {
+      if (a.fb_list && lane == 0) {
         const int pos = atomicAdd(a.fb_count, 1);
         a.fb_list[pos] = static_cast<int32_t>(n);
       }
+      return false;
+    }
+    // the winner's row again (cheaper than keeping the best candidate row live in registers)
+    const int64_t coff = (static_cast<int64_t>(a.l) * a.K + best_id) * a.D;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int i = lane * 4 + k * 128;
+      cbest[k] = i < a.D ? ld4<CB_BF16>(a.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  apply_row<NCH>(a, n, rv, cbest, best_id, lane);
+  return true;
+}
+
+template <bool CB_BF16, int SRC, int NCH>
+__global__ void __launch_bounds__(256, 2) rescore_fast_kernel(const RowArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gtid == 0 && a.fb_next) *a.fb_next = 0;
+  if (a.offsets) check_offsets(a, gtid, static_cast<int64_t>(gridDim.x) * blockDim.x);
+  const int64_t n = gtid >> 5;
+  if (n >= a.N) return;
+  rescore_row<CB_BF16, SRC, NCH>(a, n, lane);
+}
+
+// Exact scan of all K codewords for one queued row (all warps of the block; sr holds D doubles,
+// wbest/wid one slot per warp).  The chosen codeword is applied like an accepted rescore.
+template <bool CB_BF16, int SRC>
+__device__ __forceinline__ void fallback_row(const RowArgs &a, int64_t n, double *sr, double *wbest, int *wid,
+                                             int *chosen) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  __syncthreads();
+  for (int i = threadIdx.x * 4; i < a.D; i += blockDim.x * 4) {
+    const float4 v = ld_src4<SRC>(a.src, n * a.D + i);
+    sr[i] = v.x;
+    sr[i + 1] = v.y;
+    sr[i + 2] = v.z;
+    sr[i + 3] = v.w;
+  }
+  __syncthreads();
+  double bd = inf_d();
+  int bk = 0x7fffffff;
+  for (int k = warp; k < a.K; k += nwarps) {
+    const int64_t coff = (static_cast<int64_t>(a.l) * a.K + k) * a.D;
+    double acc = 0.0;
+    for (int i = lane * 4; i < a.D; i += 128) {
+      const float4 c = ld4<CB_BF16>(a.cb, coff + i);
+      const double e0 = sr[i] - c.x, e1 = sr[i + 1] - c.y, e2 = sr[i + 2] - c.z, e3 = sr[i + 3] - c.w;
+      acc += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+    }
+    acc = warp_sum_d(acc);
+    if (acc < bd) {
+      bd = acc;
+      bk = k;
+    }
+  }
+  if (lane == 0) {
+    wbest[warp] = bd;
+    wid[warp] = bk;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double b = wbest[0];
+    int k = wid[0];
+    for (int w = 1; w < nwarps; ++w)
+      if (wbest[w] < b || (wbest[w] == b && wid[w] < k)) {
+        b = wbest[w];
+        k = wid[w];
+      }
+    *chosen = k;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int id = *chosen;
+    if (id < 0 || id >= a.K) {  // only reachable with non-finite inputs
+      if (lane == 0) {
+        a.ids[n * a.L + a.l] = -1;
+        set_status(a.status, RVQ_ERR_ARG);
+      }
       return;
     }
-  }
-  float e2 = 0.f, q2 = 0.f;
-#pragma unroll
-  for (int k = 0; k < NCH; ++k) {
-    const int i = lane * 4 + k * 128;
-    if (i >= a.D) break;
-    float4 v = rv[k];
-    v.x -= cbest[k].x;
-    v.y -= cbest[k].y;
-    v.z -= cbest[k].z;
-    v.w -= cbest[k].w;
-    *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
-    if (!a.last) {
-      float4 q;
-      store_bf16x4(a.Rt + n * a.D + i, v, &q);
-      const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
-      e2 += ex * ex + ey * ey + ez * ez + ew * ew;
-      q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+    const int64_t coff = (static_cast<int64_t>(a.l) * a.K + id) * a.D;
+    float e2 = 0.f, q2 = 0.f;
+    for (int i = lane * 4; i < a.D; i += 128) {
+      const float4 c = ld4<CB_BF16>(a.cb, coff + i);
+      const float4 v = make_float4(static_cast<float>(sr[i]) - c.x, static_cast<float>(sr[i + 1]) - c.y,
+                                   static_cast<float>(sr[i + 2]) - c.z, static_cast<float>(sr[i + 3]) - c.w);
+      *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
+      if (!a.last) {
+        float4 q;
+        store_bf16x4(a.Rt + n * a.D + i, v, &q);
+        const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
+        e2 += ex * ex + ey * ey + ez * ez + ew * ew;
+        q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+      }
     }
+    if (!a.last) {
+      e2 = warp_sum_f(e2);
+      q2 = warp_sum_f(q2);
+      if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
+    }
+    if (lane == 0) a.ids[n * a.L + a.l] = id;
   }
-  if (!a.last) {
-    e2 = warp_sum_f(e2);
-    q2 = warp_sum_f(q2);
-    if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
-  }
-  if (lane == 0) a.ids[n * a.L + a.l] = best_id;
 }
 
 // Exact scan of all K codewords for the rows this level's rescore could not certify.
@@ -1117,83 +1258,8 @@ __global__ void __launch_bounds__(256) fallback_fast_kernel(const RowArgs a) {
   __shared__ int chosen;
   griddep_launch_dependents();
   griddep_wait();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int count = *a.fb_count;
-  for (int j = blockIdx.x; j < count; j += gridDim.x) {
-    const int64_t n = a.fb_list[j];
-    __syncthreads();
-    for (int i = threadIdx.x * 4; i < a.D; i += blockDim.x * 4) {
-      const float4 v = ld_src4<SRC>(a.src, n * a.D + i);
-      sr[i] = v.x;
-      sr[i + 1] = v.y;
-      sr[i + 2] = v.z;
-      sr[i + 3] = v.w;
-    }
-    __syncthreads();
-    double bd = inf_d();
-    int bk = 0x7fffffff;
-    for (int k = warp; k < a.K; k += 8) {
-      const int64_t coff = (static_cast<int64_t>(a.l) * a.K + k) * a.D;
-      double acc = 0.0;
-      for (int i = lane * 4; i < a.D; i += 128) {
-        const float4 c = ld4<CB_BF16>(a.cb, coff + i);
-        const double e0 = sr[i] - c.x, e1 = sr[i + 1] - c.y, e2 = sr[i + 2] - c.z, e3 = sr[i + 3] - c.w;
-        acc += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
-      }
-      acc = warp_sum_d(acc);
-      if (acc < bd) {
-        bd = acc;
-        bk = k;
-      }
-    }
-    if (lane == 0) {
-      wbest[warp] = bd;
-      wid[warp] = bk;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double b = wbest[0];
-      int k = wid[0];
-      for (int w = 1; w < 8; ++w)
-        if (wbest[w] < b || (wbest[w] == b && wid[w] < k)) {
-          b = wbest[w];
-          k = wid[w];
-        }
-      chosen = k;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const int id = chosen;
-      if (id < 0 || id >= a.K) {  // only reachable with non-finite inputs
-        if (lane == 0) {
-          a.ids[n * a.L + a.l] = -1;
-          set_status(a.status, RVQ_ERR_ARG);
-        }
-        continue;
-      }
-      const int64_t coff = (static_cast<int64_t>(a.l) * a.K + id) * a.D;
-      float e2 = 0.f, q2 = 0.f;
-      for (int i = lane * 4; i < a.D; i += 128) {
-        const float4 c = ld4<CB_BF16>(a.cb, coff + i);
-        const float4 v = make_float4(static_cast<float>(sr[i]) - c.x, static_cast<float>(sr[i + 1]) - c.y,
-                                     static_cast<float>(sr[i + 2]) - c.z, static_cast<float>(sr[i + 3]) - c.w);
-        *reinterpret_cast<float4 *>(a.R + n * a.D + i) = v;
-        if (!a.last) {
-          float4 q;
-          store_bf16x4(a.Rt + n * a.D + i, v, &q);
-          const float ex = v.x - q.x, ey = v.y - q.y, ez = v.z - q.z, ew = v.w - q.w;
-          e2 += ex * ex + ey * ey + ez * ez + ew * ew;
-          q2 += q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
-        }
-      }
-      if (!a.last) {
-        e2 = warp_sum_f(e2);
-        q2 = warp_sum_f(q2);
-        if (lane == 0) a.rowstat[n] = make_float2(__fsqrt_ru(e2), __fsqrt_ru(q2));
-      }
-      if (lane == 0) a.ids[n * a.L + a.l] = id;
-    }
-  }
+  for (int j = blockIdx.x; j < count; j += gridDim.x) fallback_row<CB_BF16, SRC>(a, a.fb_list[j], sr, wbest, wid, &chosen);
 }
 
 template <bool CB_BF16, int SRC>
@@ -1210,6 +1276,766 @@ inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blo
   return launch_pdl(fallback_fast_kernel<CB_BF16, SRC>, dim3(fb_blocks), dim3(256), fb_smem, s, ra);
 }
 
+// ---------------------------------------------------------------- all levels in one launch
+// One cooperative launch runs every level as a dataflow over row tiles:
+//
+//  * GEMM chunks.  Chunk (l, rt, j) scores row tile rt against codeword tiles [jS, (j+1)S) of
+//    level l and writes one partial top-8 list per row into slot j.  Chunks are numbered level by
+//    level, row tile by row tile, and CTA c takes chunks c, c+G, c+2G, ...  The TMA producer,
+//    MMA issuer, norm splitter and epilogue warps walk that sequence with the shared-memory ring,
+//    the TMEM buffers and the mbarrier phases carried from chunk to chunk.  Before loading chunk
+//    (l, rt, j) the producer waits until row tile rt is settled at level l-1.
+//  * Certificate tasks.  RW warps per CTA take tasks (l, rt, g) the same way (RPT rows each):
+//    once all NC chunks of (l, rt) are written they certify the rows, apply r -= C_l[id] and
+//    count the settled rows.  A row the certificate cannot settle goes to a queue whose exact
+//    scan is split into NS codeword slices that any certificate warp picks up while it would
+//    otherwise wait; the warp finishing a row's last slice reduces the slices, applies the winner
+//    and counts the row.
+//
+// Counters (zeroed by the host, all acquire/release at GPU scope):
+//   chunk_done[l][rt]  group-0 epilogue warps through a chunk of (l, rt)   (complete at 4 NC)
+//   cert_done[l][rt]   settled rows of (l, rt)                             (complete at the rows)
+// so level l+1 of a row tile starts while later row tiles of level l are still being scored,
+// and the certificate work runs under the tensor-core work.  Every wait is bounded: it gives up
+// when neither its counter nor the grid's progress word has moved for two seconds.
+// Certificate warps of the all-levels kernel for D in (512, 1024], next to 8 epilogue warps:
+// they fill the block up to 16 warps (the register budget per thread is set by the warp count
+// rounded up to a multiple of four).
+constexpr int FLOW_RW_WIDE = 5;
+constexpr int EXACT_QCAP = 1024;   // queued rows whose exact scan is split into slices
+constexpr int EXACT_NS_MAX = 256;  // codeword slices per queued row
+
+struct FlowArgs {
+  int L;
+  int64_t RT;
+  int NC, S;        // chunks per row tile, codeword tiles per chunk
+  int RPT;          // rows per certificate task (divides 128)
+  int NS, slice;    // exact-scan slices per queued row, codewords per slice
+  uint32_t *chunk_done;  // [L, RT]
+  uint32_t *cert_done;   // [L, RT]
+  uint32_t *ctr;         // queued rows, next slice, settled rows, progress
+  int4 *ex_entry;        // [EXACT_QCAP]: row, level, ready flag, slices done
+  double2 *ex_part;      // [EXACT_QCAP, NS]: best distance of a slice, its codeword id
+  int32_t *fb_level;     // [L] rows per level that took the exact scan
+  const float *norms;    // [L, K]
+  const float *level_stats;
+};
+
+// Wait until *ctr >= target (acquire).  Gives up, sets *abort and returns false when neither
+// *ctr nor the grid's progress word has moved for limit_ns.
+__device__ __noinline__ bool wait_count(const uint32_t *ctr, uint32_t target, const uint32_t *progress,
+                                        volatile int *abort, uint64_t limit_ns = 2000000000ull) {
+  uint32_t c = ld_acquire_gpu(ctr);
+  if (c >= target) return true;
+  uint32_t last_c = c;
+  uint32_t last_p = *reinterpret_cast<const volatile uint32_t *>(progress);
+  uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(100);
+    c = ld_acquire_gpu(ctr);
+    if (c >= target) return true;
+    if (*abort) return false;
+    const uint32_t pr = *reinterpret_cast<const volatile uint32_t *>(progress);
+    const uint64_t now = global_timer_ns();
+    if (c != last_c || pr != last_p) {
+      last_c = c;
+      last_p = pr;
+      t0 = now;
+    } else if (now - t0 > limit_ns) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Publish this warp's global writes and add v (warp-uniform) to *ctr.  TMA: the writes are also
+// made visible to the async proxy (later TMA loads of the residual operand).
+template <bool TMA>
+__device__ __forceinline__ void warp_release_add(uint32_t *ctr, uint32_t v, int lane) {
+  if constexpr (TMA) fence_proxy_async_global();
+  __syncwarp();
+  if (lane == 0 && v) red_release_add_gpu(ctr, v);
+}
+
+// Exact scan of all K codewords of level a.l for row n by one warp (slow path, used only when
+// the slice queue is full): lane j scores codewords j, j+32, ... with fp64 accumulation of fp32
+// differences, the residual row broadcast from the registers that hold it; lowest index on
+// ties.  Applies the winner like an accepted rescore.
+template <bool CB_BF16, int SRC, int NCH>
+__device__ __noinline__ void exact_row(const RowArgs &a, int64_t n, int lane) {
+  float4 rv[NCH];
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    rv[k] = i < a.D ? ld_src4<SRC>(a.src, n * a.D + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int64_t lvl = static_cast<int64_t>(a.l) * a.K;
+  double best = inf_d();
+  int bid = 0x7fffffff;
+  for (int k0 = 0; k0 < a.K; k0 += 32) {
+    const int k = k0 + lane;
+    const int64_t coff = (lvl + (k < a.K ? k : a.K - 1)) * a.D;
+    double acc = 0.0;
+#pragma unroll
+    for (int q = 0; q < NCH; ++q) {
+#pragma unroll 4
+      for (int s = 0; s < 32; ++s) {
+        if (q * 128 + s * 4 >= a.D) break;
+        const float rx = __shfl_sync(0xffffffffu, rv[q].x, s), ry = __shfl_sync(0xffffffffu, rv[q].y, s);
+        const float rz = __shfl_sync(0xffffffffu, rv[q].z, s), rw = __shfl_sync(0xffffffffu, rv[q].w, s);
+        const float4 c = ld4<CB_BF16>(a.cb, coff + q * 128 + s * 4);
+        const double e0 = static_cast<double>(rx) - c.x, e1 = static_cast<double>(ry) - c.y;
+        const double e2 = static_cast<double>(rz) - c.z, e3 = static_cast<double>(rw) - c.w;
+        acc += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+      }
+    }
+    if (k < a.K && acc < best) {
+      best = acc;
+      bid = k;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bid, off);
+    if (ob < best || (ob == best && oi < bid)) {
+      best = ob;
+      bid = oi;
+    }
+  }
+  if (bid < 0 || bid >= a.K) {  // only reachable with non-finite inputs
+    if (lane == 0) {
+      a.ids[n * a.L + a.l] = -1;
+      set_status(a.status, RVQ_ERR_ARG);
+    }
+    return;
+  }
+  float4 c[NCH];
+  const int64_t coff = (lvl + bid) * a.D;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    c[k] = i < a.D ? ld4<CB_BF16>(a.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  apply_row<NCH>(a, n, rv, c, bid, lane);
+}
+
+// One slice of a queued row's exact scan: codewords [k0, k1) of level a.l, one codeword per
+// warp step (coalesced rows), UNR codewords in flight; fp64 accumulation of fp32 differences,
+// lowest index on ties.  Returns the slice's best distance and codeword in every lane.
+template <bool CB_BF16, int NCH>
+__device__ __forceinline__ void exact_slice(const RowArgs &a, int64_t n, int k0, int k1, const float4 (&rv)[NCH],
+                                            int lane, double &best, int &bid) {
+  constexpr int UNR = NCH <= 2 ? 4 : NCH <= 4 ? 2 : 1;
+  const int64_t lvl = static_cast<int64_t>(a.l) * a.K;
+  best = inf_d();
+  bid = 0x7fffffff;
+  for (int k = k0; k < k1; k += UNR) {
+    double acc[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int kk = k + u < k1 ? k + u : k1 - 1;
+      const int64_t coff = (lvl + kk) * a.D;
+      float4 c[NCH];
+#pragma unroll
+      for (int q = 0; q < NCH; ++q) {
+        const int i = lane * 4 + q * 128;
+        c[q] = i < a.D ? ld4<CB_BF16>(a.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      double s = 0.0;
+#pragma unroll
+      for (int q = 0; q < NCH; ++q) {
+        const double e0 = static_cast<double>(rv[q].x) - c[q].x, e1 = static_cast<double>(rv[q].y) - c[q].y;
+        const double e2 = static_cast<double>(rv[q].z) - c[q].z, e3 = static_cast<double>(rv[q].w) - c[q].w;
+        s += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+      }
+      acc[u] = s;
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const double d = warp_sum_d(acc[u]);
+      if (k + u < k1 && d < best) {
+        best = d;
+        bid = k + u;
+      }
+    }
+  }
+}
+
+template <int EPI, int RW>
+struct FlowCfg {
+  static constexpr int THREADS = GemmCfg<EPI, false>::THREADS + RW * 32;
+  static constexpr int CERT0 = EPI + 3;  // first certificate warp
+};
+
+template <int EPI, int RW, bool CB_BF16, bool X_BF16, int NCH>
+__global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
+    encode_flow_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB3, const GemmArgs a, const RowArgs r0,
+                       const FlowArgs fa) {
+  using C = GemmCfg<EPI, false>;
+  constexpr int NSTAGE = C::NSTAGE;
+  constexpr int CERT0 = FlowCfg<EPI, RW>::CERT0;
+  constexpr int SRC0 = X_BF16 ? SRC_X_BF16 : SRC_X_F32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *aug_a = smem + C::AUG_A_OFF;
+  uint8_t *aug_b = smem + C::AUG_B_OFF;
+  float2 *mbuf = reinterpret_cast<float2 *>(smem + C::MERGE_OFF);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  uint64_t *empty = full + NSTAGE;
+  uint64_t *tfull = empty + NSTAGE;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *afull = tempty + 2;
+  uint64_t *mready = afull + 2;
+  uint64_t *mdone = mready + 1;
+  uint64_t *mma_done = mdone + 1;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  volatile int *never = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = a.D / BK;
+  const uint32_t G = gridDim.x;
+  const int64_t RT = fa.RT;
+  const int64_t total_chunks = static_cast<int64_t>(fa.L) * RT * fa.NC;
+  uint32_t *ex_rows = fa.ctr;
+  uint32_t *ex_next = fa.ctr + 1;
+  uint32_t *settled = fa.ctr + 2;
+  uint32_t *progress = fa.ctr + 3;
+  // rows of row tile rt (the last tile may be short)
+  auto tile_rows = [&](int64_t rt) -> uint32_t {
+    return static_cast<uint32_t>(min(static_cast<int64_t>(BM), a.N - rt * BM));
+  };
+  // First codeword tile this CTA visits in a chunk of cnt tiles: CTAs spread their starting
+  // points over the chunk so they do not all stream the same codeword tile at the same time.
+  auto chunk_rot = [&](int cnt) -> int { return static_cast<int>((static_cast<int64_t>(blockIdx.x) * cnt) / G); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::EPI_THREADS);
+      mbar_init(&afull[b], 32);
+    }
+    mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
+    mbar_init(mdone, 128);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < (AUG_A_BYTES + 2 * AUG_B_BYTES) / 16; i += blockDim.x) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (i < AUG_A_BYTES / 16 && ((i * 16) % 256) < 128)
+      v = make_uint4(BF16_ONE | (static_cast<uint32_t>(BF16_ONE) << 16), BF16_ONE, 0, 0);
+    reinterpret_cast<uint4 *>(aug_a)[i] = v;
+  }
+  fence_proxy_async_smem();
+  if (warp == C::ISSUER) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  int p_s = 0;  // producer ring position, kept for the teardown
+  uint32_t p_ph = 0;
+  int64_t p_issued = 0;
+
+  if (warp == C::PRODUCER) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA0);
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB3);
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+        const int j = static_cast<int>(t % fa.NC);
+        const int64_t rt = (t / fa.NC) % RT;
+        const int l = static_cast<int>(t / (fa.NC * RT));
+        if (l > 0) {
+          if (!wait_count(fa.cert_done + (l - 1) * RT + rt, tile_rows(rt), progress, abort_flag)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // residual rows written by the generic proxy, read by TMA
+        }
+        const CUtensorMap *mA = l == 0 ? &tmA0 : &tmA;
+        const int ct0 = j * fa.S, cnt = min(a.Tc, ct0 + fa.S) - ct0;
+        const int rot = chunk_rot(cnt);
+        for (int k = 0; k < cnt && ok; ++k) {
+          const int ct = ct0 + (rot + k) % cnt;
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&empty[p_s], p_ph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[p_s], C::STAGE);
+            uint8_t *sa = smem + p_s * C::STAGE;
+            tma_load_2d(mA, &full[p_s], sa, kb * BK, static_cast<int32_t>(rt * BM));
+            tma_load_3d(&tmB3, &full[p_s], sa + A_BYTES, kb * BK, ct * BN, l);
+            ++p_issued;
+            if (++p_s == NSTAGE) {
+              p_s = 0;
+              p_ph ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(a.status, RVQ_ERR_TIMEOUT);
+      }
+    }
+  } else if (warp == C::SPLITTER) {
+    // ------------------------------------------------------------ norm split -> B_aug tiles
+    int64_t i = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+      const int j = static_cast<int>(t % fa.NC);
+      const int l = static_cast<int>(t / (fa.NC * RT));
+      const float *norms_l = fa.norms + static_cast<int64_t>(l) * a.K;
+      const int ct0 = j * fa.S, cnt = min(a.Tc, ct0 + fa.S) - ct0;
+      const int rot = chunk_rot(cnt);
+      for (int k = 0; k < cnt; ++k, ++i) {
+        const int ct = ct0 + (rot + k) % cnt;
+        const int slot = static_cast<int>(i & 1);
+        const int c0 = ct * BN + lane * 8;
+        float hv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) hv[q] = c0 + q < a.K ? 0.5f * __ldg(norms_l + c0 + q) : 0.f;
+        bool got = i < 2 || mbar_wait(&tfull[slot], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(aug_b + slot * AUG_B_BYTES + lane * 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint16_t h1, h2 = 0, h3 = 0;
+          if (c0 + q < a.K) {
+            h1 = bf16_bits_rn(hv[q]);
+            const float r1 = hv[q] - bf16_bits_to_float(h1);
+            h2 = bf16_bits_rn(r1);
+            const float r2 = r1 - bf16_bits_to_float(h2);
+            h3 = bf16_bits_rn(r2);
+          } else {
+            h1 = BF16_BIG;
+          }
+          dst[q] = make_uint4(h1 | (static_cast<uint32_t>(h2) << 16), h3, 0, 0);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&afull[slot]);
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(a.status, RVQ_ERR_TIMEOUT);
+    }
+  } else if (warp == C::ISSUER) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main = idesc_bf16_f32(BM, BN, true);
+      constexpr uint32_t idesc_aug = idesc_bf16_f32(BM, BN, false);
+      const uint64_t adesc_aug = sdesc_k_noswizzle(smem_u32(aug_a), 128, 256);
+      int m_s = 0;
+      uint32_t m_ph = 0;
+      int64_t i = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+        const int j = static_cast<int>(t % fa.NC);
+        const int cnt = min(a.Tc, j * fa.S + fa.S) - j * fa.S;
+        for (int k = 0; k < cnt && ok; ++k, ++i) {
+          const int buf = static_cast<int>(i & 1);
+          const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
+          if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag) || !mbar_wait(&afull[buf], tph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
+          umma_f16(dt, adesc_aug, sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128), idesc_aug, 0u);
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[m_s], m_ph, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + m_s * C::STAGE);
+            const uint64_t ad = sdesc_k128(sa);
+            const uint64_t bd = sdesc_k128(sa + A_BYTES);
+#pragma unroll
+            for (int k = 0; k < BK / UK; ++k) {
+              const uint64_t step = static_cast<uint64_t>(k * UK * 2 / 16);
+              umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
+            }
+            umma_commit(&empty[m_s]);
+            if (++m_s == NSTAGE) {
+              m_s = 0;
+              m_ph ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&tfull[buf]);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(a.status, RVQ_ERR_TIMEOUT);
+      }
+    }
+  } else if (warp < EPI) {
+    // ------------------------------------------------------------ epilogue: running top-8 per chunk
+    const int quad = warp & 3;
+    const int grp = warp >> 2;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    float bd[TOPK];
+    int bi[TOPK];
+    int64_t i = 0;
+    uint32_t nflush = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+      const int j = static_cast<int>(t % fa.NC);
+      const int64_t rt = (t / fa.NC) % RT;
+      const int l = static_cast<int>(t / (fa.NC * RT));
+#pragma unroll
+      for (int q = 0; q < TOPK; ++q) {
+        bd[q] = inf_f();
+        bi[q] = -1;
+      }
+      // slot j of (l-1, rt) must have been read by every certificate task before it is rewritten:
+      // the producer already waited for that, so this load (checked at the flush) only orders it
+      uint32_t settled_prev = 0xffffffffu;
+      if (grp == 0 && lane == 0 && l > 0) settled_prev = ld_acquire_gpu(fa.cert_done + (l - 1) * RT + rt);
+      const int ct0 = j * fa.S, cnt = min(a.Tc, ct0 + fa.S) - ct0;
+      const int rot = chunk_rot(cnt);
+      for (int k = 0; k < cnt; ++k, ++i) {
+        const int ct = ct0 + (rot + k) % cnt;
+        const int buf = static_cast<int>(i & 1);
+        const uint32_t tph = static_cast<uint32_t>((i >> 1) & 1);
+        const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int col0 = ct * BN;
+        const int nvalid = min(BN, a.K - col0);
+#pragma unroll 1
+        for (int ch = 0; ch < C::CHUNKS; ++ch) {
+          const int ct0 = grp * C::COLS + ch * 32;
+          uint32_t vv[32];
+          tmem_ld_32x32(lane_base + static_cast<uint32_t>(buf * BN + ct0), vv);
+          tmem_ld_wait();
+          if (ch == C::CHUNKS - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int c0 = col0 + ct0;
+          float d[32];
+          if (ct0 + 32 <= nvalid) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) d[q] = __uint_as_float(vv[q]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) d[q] = (ct0 + q < nvalid) ? __uint_as_float(vv[q]) : kPastK;
+          }
+          float m11[11];
+#pragma unroll
+          for (int q = 0; q < 10; ++q) m11[q] = fmin3(d[3 * q], d[3 * q + 1], d[3 * q + 2]);
+          m11[10] = fminf(d[30], d[31]);
+          const float m4a = fmin3(m11[0], m11[1], m11[2]), m4b = fmin3(m11[3], m11[4], m11[5]);
+          const float m4c = fmin3(m11[6], m11[7], m11[8]), m4d = fminf(m11[9], m11[10]);
+          const float m = fminf(fmin3(m4a, m4b, m4c), m4d);
+          const unsigned need = __ballot_sync(0xffffffffu, m < bd[TOPK - 1]);
+          if (__popc(need) >= kMergeLanes) {
+            topk_merge_chunk(bd, bi, d, c0);
+          } else if (need) {
+            topk_insert_few(bd, bi, d, c0);
+          }
+        }
+      }
+      if (!ok) break;
+      // ---- flush: merge the column groups, write slot j of row tile rt
+      if constexpr (C::GROUPS > 1) {
+        float2 *mine = mbuf + (static_cast<int64_t>(grp - 1) * BM + row_in_tile) * TOPK;
+        if (grp > 0) {
+          if (nflush > 0 && !mbar_wait(mdone, (nflush - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int q = 0; q < TOPK; ++q) mine[q] = make_float2(bd[q], __int_as_float(bi[q]));
+          mbar_arrive(mready);
+        } else {
+          if (!mbar_wait(mready, nflush & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          #pragma unroll 1
+          for (int e8 = 0; e8 < (C::GROUPS - 1) * TOPK; ++e8) {
+            const float2 e = mbuf[(static_cast<int64_t>(e8 / TOPK) * BM + row_in_tile) * TOPK + e8 % TOPK];
+            if (e.x < bd[TOPK - 1]) topk_insert(bd, bi, e.x, __float_as_int(e.y));
+          }
+          mbar_arrive(mdone);
+        }
+      }
+      ++nflush;
+      if (grp == 0) {
+        // the slot is rewritten only after every certificate task of (l-1, rt) has read it
+        bool got = true;
+        if (lane == 0 && settled_prev < tile_rows(rt))
+          got = wait_count(fa.cert_done + (l - 1) * RT + rt, tile_rows(rt), progress, abort_flag);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const int64_t n = rt * BM + row_in_tile;
+        if (n < a.N) {
+          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + j) * BM + row_in_tile) * TOPK);
+#pragma unroll
+          for (int q = 0; q < TOPK; ++q)
+            if (bi[q] >= a.K) {
+              bd[q] = inf_f();
+              bi[q] = -1;
+            }
+#pragma unroll
+          for (int q = 0; q < TOPK; q += 2)
+            out[q / 2] = make_float4(2.f * bd[q], __int_as_float(bi[q]), 2.f * bd[q + 1], __int_as_float(bi[q + 1]));
+        }
+        warp_release_add<false>(fa.chunk_done + static_cast<int64_t>(l) * RT + rt, 1u, lane);
+        if (warp == 0 && lane == 0) atomicAdd(progress, 1u);  // liveness for the bounded waits
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(a.status, RVQ_ERR_TIMEOUT);
+    }
+  } else if (warp >= CERT0) {
+    // ------------------------------------------------------------ certificate warps
+    const int64_t cw = static_cast<int64_t>(G) * RW;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * RW + (warp - CERT0);
+    const int TG = BM / fa.RPT;
+    const int64_t total_tasks = static_cast<int64_t>(fa.L) * RT * TG;
+    const uint32_t all_rows = static_cast<uint32_t>(a.N) * static_cast<uint32_t>(fa.L);
+    RowArgs ra = r0;  // r0.nslots = NC: a row tile's candidate lists are its chunks' slots
+    bool ok = true;
+
+    // Claim and run one slice of a queued row's exact scan; false when none is ready.
+    auto help_exact = [&]() -> bool {
+      int64_t claimed = -1;
+      int en = 0, el = 0;
+      if (lane == 0) {
+        const uint32_t s = ld_acquire_gpu(ex_next);
+        const uint32_t rows = min(ld_acquire_gpu(ex_rows), static_cast<uint32_t>(EXACT_QCAP));
+        if (s < rows * static_cast<uint32_t>(fa.NS)) {
+          const int q = static_cast<int>(s / fa.NS);
+          if (ld_acquire_gpu(reinterpret_cast<const uint32_t *>(&fa.ex_entry[q].z)) != 0 &&
+              atomicCAS(ex_next, s, s + 1) == s) {
+            claimed = s;
+            const int4 e = __ldcg(fa.ex_entry + q);
+            en = e.x;
+            el = e.y;
+          }
+        }
+      }
+      claimed = __shfl_sync(0xffffffffu, claimed, 0);
+      if (claimed < 0) return false;
+      const int q = static_cast<int>(claimed / fa.NS), sl = static_cast<int>(claimed % fa.NS);
+      const int64_t n = __shfl_sync(0xffffffffu, en, 0);
+      const int l = __shfl_sync(0xffffffffu, el, 0);
+      RowArgs xa = r0;
+      xa.l = l;
+      xa.last = l == fa.L - 1;
+      xa.src = l == 0 ? r0.src : static_cast<const void *>(r0.R);
+      float4 rv[NCH];
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        const int i = lane * 4 + k * 128;
+        rv[k] = i >= a.D ? make_float4(0.f, 0.f, 0.f, 0.f)
+                : l == 0 ? ld_src4<SRC0>(xa.src, n * a.D + i) : ld_src4<SRC_R>(xa.src, n * a.D + i);
+      }
+      const int k0 = sl * fa.slice, k1 = min(a.K, k0 + fa.slice);
+      double best;
+      int bid;
+      exact_slice<CB_BF16, NCH>(xa, n, k0, k1, rv, lane, best, bid);
+      uint32_t old = 0;
+      if (lane == 0) {
+        fa.ex_part[static_cast<int64_t>(q) * fa.NS + sl] = make_double2(best, static_cast<double>(bid));
+        __threadfence();
+        old = atomicAdd(reinterpret_cast<uint32_t *>(&fa.ex_entry[q].w), 1u);
+        __threadfence();
+        atomicAdd(progress, 1u);
+      }
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old + 1 == static_cast<uint32_t>(fa.NS)) {
+        // last slice: reduce (lowest distance, then lowest index) and settle the row
+        double b = inf_d();
+        int id = 0x7fffffff;
+        for (int s2 = lane; s2 < fa.NS; s2 += 32) {
+          const double2 pr = __ldcg(fa.ex_part + static_cast<int64_t>(q) * fa.NS + s2);
+          const int pid = static_cast<int>(pr.y);
+          if (pr.x < b || (pr.x == b && pid < id)) {
+            b = pr.x;
+            id = pid;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+          const double ob = __shfl_xor_sync(0xffffffffu, b, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, id, off);
+          if (ob < b || (ob == b && oi < id)) {
+            b = ob;
+            id = oi;
+          }
+        }
+        if (id < 0 || id >= a.K) {  // only reachable with non-finite inputs
+          if (lane == 0) {
+            r0.ids[n * r0.L + l] = -1;
+            set_status(a.status, RVQ_ERR_ARG);
+          }
+        } else {
+          float4 c[NCH];
+          const int64_t coff = (static_cast<int64_t>(l) * a.K + id) * a.D;
+#pragma unroll
+          for (int k = 0; k < NCH; ++k) {
+            const int i = lane * 4 + k * 128;
+            c[k] = i < a.D ? ld4<CB_BF16>(r0.cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          apply_row<NCH>(xa, n, rv, c, id, lane);
+        }
+        warp_release_add<true>(fa.cert_done + static_cast<int64_t>(l) * RT + n / BM, 1u, lane);
+        if (lane == 0) atomicAdd(settled, 1u);
+      }
+      return true;
+    };
+    // Wait for *ctr >= target, running exact-scan slices meanwhile.
+    auto wait_helping = [&](const uint32_t *ctr, uint32_t target) -> bool {
+      uint32_t last_p = 0;
+      uint64_t t0 = 0;
+      bool first = true;
+      while (true) {
+        uint32_t c = 0, pr = 0;
+        if (lane == 0) {
+          c = ld_acquire_gpu(ctr);
+          pr = *reinterpret_cast<const volatile uint32_t *>(progress);
+        }
+        c = __shfl_sync(0xffffffffu, c, 0);
+        if (c >= target) return true;
+        if (*abort_flag) return false;
+        if (help_exact()) {
+          first = true;
+          continue;
+        }
+        pr = __shfl_sync(0xffffffffu, pr, 0);
+        const uint64_t now = global_timer_ns();
+        if (first || pr != last_p) {
+          first = false;
+          last_p = pr;
+          t0 = now;
+        } else if (now - t0 > 2000000000ull) {
+          *abort_flag = 1;
+          return false;
+        }
+        __nanosleep(200);
+      }
+    };
+
+    for (int64_t s = gw; s < total_tasks && ok; s += cw) {
+      const int g = static_cast<int>(s % TG);
+      const int64_t rt = (s / TG) % RT;
+      const int l = static_cast<int>(s / (TG * RT));
+      if (!wait_helping(fa.chunk_done + static_cast<int64_t>(l) * RT + rt, 4u * fa.NC) ||
+          (l > 0 && !wait_helping(fa.cert_done + static_cast<int64_t>(l - 1) * RT + rt, tile_rows(rt)))) {
+        ok = false;
+        break;
+      }
+      ra.l = l;
+      ra.last = l == fa.L - 1;
+      ra.stats = fa.level_stats + static_cast<int64_t>(l) * RVQ_LEVEL_STATS;
+      ra.src = l == 0 ? r0.src : static_cast<const void *>(r0.R);
+      if (l == 0 && rt == 0 && g == 0 && r0.offsets) check_offsets(ra, lane, 32);
+      const int64_t n0 = rt * BM + static_cast<int64_t>(g) * fa.RPT;
+      const int64_t n1 = min(a.N, n0 + fa.RPT);
+      uint32_t done_rows = 0;
+      for (int64_t n = n0; n < n1; ++n) {
+        const bool settled_row = l == 0 ? rescore_row<CB_BF16, SRC0, NCH>(ra, n, lane)
+                                        : rescore_row<CB_BF16, SRC_R, NCH>(ra, n, lane);
+        if (settled_row) {
+          ++done_rows;
+          continue;
+        }
+        // queue the row's exact scan (or, with the queue full, scan it here)
+        uint32_t q = 0;
+        if (lane == 0) {
+          q = atomicAdd(ex_rows, 1u);
+          atomicAdd(fa.fb_level + l, 1);
+          if (q < EXACT_QCAP) {
+            fa.ex_entry[q] = make_int4(static_cast<int>(n), l, 0, 0);
+            __threadfence();
+            atomicExch(reinterpret_cast<uint32_t *>(&fa.ex_entry[q].z), 1u);
+          }
+        }
+        q = __shfl_sync(0xffffffffu, q, 0);
+        if (q >= EXACT_QCAP) {
+          if (l == 0)
+            exact_row<CB_BF16, SRC0, NCH>(ra, n, lane);
+          else
+            exact_row<CB_BF16, SRC_R, NCH>(ra, n, lane);
+          ++done_rows;
+        }
+      }
+      warp_release_add<true>(fa.cert_done + static_cast<int64_t>(l) * RT + rt, done_rows, lane);
+      if (lane == 0) {
+        if (done_rows) atomicAdd(settled, done_rows);
+        atomicAdd(progress, 1u);
+      }
+    }
+    // help with the remaining exact scans until every row of every level is settled
+    if (ok && !wait_helping(settled, all_rows)) ok = false;
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(a.status, RVQ_ERR_TIMEOUT);
+    }
+  }
+
+  // no bulk copy or MMA may still be in flight when the block exits
+  if (warp == C::ISSUER && lane == 0) {
+    umma_commit(mma_done);
+    mbar_wait(mma_done, 0, never);
+  }
+  if (warp == C::PRODUCER && lane == 0 && *abort_flag) {
+    const int64_t pending = p_issued < NSTAGE ? p_issued : NSTAGE;
+    for (int64_t jj = 0; jj < pending; ++jj) {
+      int back = p_s - 1 - static_cast<int>(jj);
+      uint32_t ph = p_ph;
+      while (back < 0) {
+        back += NSTAGE;
+        ph ^= 1u;
+      }
+      mbar_wait(&full[back], ph, never);
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::ISSUER) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host plan
 
 struct Plan {
@@ -1217,9 +2043,35 @@ struct Plan {
   int Tc;
   int64_t U;
   int G;       // CTAs, or CTA pairs when pair
-  int maxs;
+  int maxs;    // partial-list slots per row tile (the larger of the two paths' needs)
   bool pair;
+  // all levels in one cooperative launch (encode_flow_kernel)
+  bool flow;
+  int L;
+  int NC, S;      // chunks per row tile, codeword tiles per chunk
+  int RPT;        // rows per certificate task
+  int NS, slice;  // exact-scan slices per queued row, codewords per slice
+  int Gf;         // CTAs of the flow launch (one per SM)
 };
+
+// RVQ_PERSISTENT=0 keeps the per-level launches for every width (tuning / comparison knob).
+inline bool persistent_enabled() {
+  static int v = [] {
+    const char *e = getenv("RVQ_PERSISTENT");
+    return e ? atoi(e) : 1;
+  }();
+  return v != 0;
+}
+
+// Row chunks (float4 per lane) of the register-resident row kernels for feature width D <= 1024.
+inline int row_chunks(int D) { return D <= 128 ? 1 : D <= 256 ? 2 : D <= 512 ? 4 : 8; }
+
+// Slots a row tile of Tc units needs when U units are split into G ranges: every range but the
+// last holds at least f = floor(U/G) units, so Tc consecutive units meet at most 1 + ceil((Tc-1)/f).
+inline int64_t slots_needed(int64_t U, int64_t G, int64_t Tc) {
+  const int64_t f = std::max<int64_t>(1, U / G);
+  return std::min<int64_t>(G, 1 + (Tc - 1 + f - 1) / f);
+}
 
 // CTA pairs (tcgen05 cta_group::2) halve the codeword traffic per SM.  Off unless RVQ_PAIR=1
 // (tuning knob): on the measured workloads the single-CTA kernel is not L2-bound.
@@ -1233,7 +2085,8 @@ inline bool use_pairs(int64_t N) {
 
 int resident_pair_clusters(int D);
 
-inline Plan make_plan(int64_t N, int K, int D, int sms) {
+inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
+  const int sms0 = sms;
   Plan p;
   p.pair = use_pairs(N);
   if (p.pair) {
@@ -1254,15 +2107,38 @@ inline Plan make_plan(int64_t N, int K, int D, int sms) {
   int64_t G = std::min<int64_t>(sms, p.U);
   G = std::min<int64_t>(G, std::max<int64_t>(1, p.U / need_f));
   p.G = static_cast<int>(G);
-  const int64_t f = p.U / p.G;
-  p.maxs = static_cast<int>(std::min<int64_t>(p.G, 1 + (p.Tc - 1 + f - 1) / f));
+  p.maxs = static_cast<int>(slots_needed(p.U, p.G, p.Tc));
+
+  const int nch = row_chunks(D);
+  p.L = L;
+  // D in (512, 1024] only: at D <= 256 the distance epilogue is issue-bound and leaves the block
+  // room for one certificate warp, which cannot keep up (measured), so levels run one by one
+  p.flow = !p.pair && D <= 1024 && nch == 8 && persistent_enabled() &&
+           static_cast<uint64_t>(N) * static_cast<uint64_t>(L) < (uint64_t(1) << 32);
+  p.NC = p.S = p.RPT = p.NS = p.slice = p.Gf = 0;
+  if (p.flow) {
+    p.Gf = sms0;
+    // enough chunks per level to keep every CTA busy and finish a row tile soon after it starts
+    int nc = static_cast<int>(std::min<int64_t>(MAX_SLOTS, std::max<int64_t>(1, (4 * p.Gf + p.RT - 1) / p.RT)));
+    nc = std::min(nc, p.Tc);
+    p.S = (p.Tc + nc - 1) / nc;
+    p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
+    p.maxs = std::max(p.maxs, p.NC);
+    // certificate tasks: about two per certificate warp per level, at most one row tile each
+    const int64_t cw = static_cast<int64_t>(p.Gf) * FLOW_RW_WIDE;
+    int tg = 1;
+    while (tg < 64 && static_cast<int64_t>(tg) * p.RT < 2 * cw) tg *= 2;
+    p.RPT = BM / tg;
+    p.slice = std::max(64, (K + EXACT_NS_MAX - 1) / EXACT_NS_MAX);
+    p.NS = (K + p.slice - 1) / p.slice;
+  }
   return p;
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t R, Rt, rowstat, cand, fb_list, fb_count, total;
+  size_t R, Rt, rowstat, cand, fb_list, fb_count, sync, sync_end, ex_part, total;
 };
 
 inline Layout make_layout(int64_t N, int D, const Plan &p) {
@@ -1280,6 +2156,13 @@ inline Layout make_layout(int64_t N, int D, const Plan &p) {
   off += align256(static_cast<size_t>(N) * 4);
   w.fb_count = off;
   off += align256(64 * 4);
+  w.sync = off;  // directly after fb_count: one memset clears both
+  if (p.flow) {  // progress counters, chunk_done [L, RT], cert_done [L, RT], exact-scan queue entries
+    off += 256 + align256(2 * static_cast<size_t>(p.L) * p.RT * 4) + align256(EXACT_QCAP * 16);
+  }
+  w.sync_end = off;
+  w.ex_part = off;
+  if (p.flow) off += align256(static_cast<size_t>(EXACT_QCAP) * p.NS * 16);
   w.total = off;
   return w;
 }
@@ -1299,6 +2182,19 @@ inline EncodeTiledFn encode_tiled_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
+}
+
+// bf16 [L, K, D] row-major as a 3-D tensor, box = BK x box_rows x 1, 128B swizzle.
+inline bool make_map3(CUtensorMap *m, const void *base, int L, int K, int D, int box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(L)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(K) * D * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 [rows, D] row-major, box = BK elements x box_rows rows, 128B swizzle, zero fill outside.
@@ -1396,6 +2292,52 @@ inline int resident_pair_clusters(int D) {
   return epi == 4 ? max_pair_clusters<4>() : epi == 16 ? max_pair_clusters<16>() : max_pair_clusters<8>();
 }
 
+// All-levels dataflow encode, instantiated for D in (512, 1024] (see FLOW_RW_WIDE).
+
+template <int EPI, int RW, bool CB, bool XB, int NCH>
+inline bool set_flow_attr() {
+  return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, CB, XB, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<EPI, false>::SMEM) == cudaSuccess;
+}
+
+inline bool flow_attrs_ready() {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] {
+    constexpr int RWD = FLOW_RW_WIDE;
+    ok = set_flow_attr<8, RWD, false, false, 8>() && set_flow_attr<8, RWD, false, true, 8>() &&
+         set_flow_attr<8, RWD, true, false, 8>() && set_flow_attr<8, RWD, true, true, 8>();
+  });
+  return ok;
+}
+
+template <int EPI, int RW, bool CB, bool XB, int NCH>
+inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tmA0, const CUtensorMap &tmA,
+                                 const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(FlowCfg<EPI, RW>::THREADS);
+  cfg.dynamicSmemBytes = GemmCfg<EPI, false>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: CTAs wait on one another's counters
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, CB, XB, NCH>, tmA0, tmA, tmB3, ga, ra, fa);
+}
+
+inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cudaStream_t s, const CUtensorMap &tmA0,
+                               const CUtensorMap &tmA, const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra,
+                               const FlowArgs &fa) {
+  constexpr int RWD = FLOW_RW_WIDE;
+  if (nch != 8) return cudaErrorInvalidValue;
+  if (cb_bf16) return x_bf16 ? launch_flow_t<8, RWD, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                             : launch_flow_t<8, RWD, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  return x_bf16 ? launch_flow_t<8, RWD, false, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                : launch_flow_t<8, RWD, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+}
+
 inline cudaError_t launch_gemm(int epi, bool pair, int groups, cudaStream_t s, const CUtensorMap &tmA,
                                const CUtensorMap &tmB, const GemmArgs &ga) {
   if (pair) {
@@ -1418,7 +2360,7 @@ extern "C" int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t 
   int sms = 0;
   int st = device_sm_count(&sms);
   if (st != RVQ_OK) return st;
-  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, sms);
+  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, L, sms);
   *bytes = enc::make_layout(N, D, p).total;
   return RVQ_OK;
 }
@@ -1446,7 +2388,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   int sms = 0;
   int st = device_sm_count(&sms);
   if (st != RVQ_OK) return st;
-  const Plan p = make_plan(N, K, D, sms);
+  const Plan p = make_plan(N, K, D, L, sms);
   const Layout w = make_layout(N, D, p);
   if (workspace_bytes < w.total) return RVQ_ERR_WORKSPACE;
 
@@ -1469,7 +2411,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   // are their own tensor-core operand, so no initial copy at all).  Wider rows: the init kernel
   // materialises the fp32 residual and the row kernels stream it.
   const bool fast = D <= 1024;
-  const int nch = D <= 128 ? 1 : D <= 256 ? 2 : D <= 512 ? 4 : 8;
+  const int nch = row_chunks(D);
   const bool x_is_operand = fast && f_dtype == RVQ_BF16;
   if (!x_is_operand) {
     const int64_t threads = N * 32;
@@ -1490,10 +2432,82 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   CUtensorMap tmX;
   if (x_is_operand && !make_map(&tmX, features, N, D, BM)) return RVQ_ERR_CUDA;
 
+  // D in (128, 256] or (512, 1024]: every level in one cooperative launch.
+  const bool all_levels = fast && p.flow;
+  if (all_levels) {
+    if (!flow_attrs_ready()) return RVQ_ERR_CUDA;
+    CUtensorMap tmB3;
+    if (!make_map3(&tmB3, op, L, K, D, BN)) return RVQ_ERR_CUDA;
+    if (cudaMemsetAsync(fb_count, 0, w.sync_end - w.fb_count, s) != cudaSuccess) return RVQ_ERR_CUDA;
+    uint8_t *sync = ws + w.sync;
+    GemmArgs ga;
+    ga.norms = norms;
+    ga.N = N;
+    ga.K = K;
+    ga.D = D;
+    ga.U = 0;  // chunks, not unit ranges: FlowArgs
+    ga.Tc = p.Tc;
+    ga.G = p.Gf;
+    ga.maxs = p.maxs;
+    ga.cand = cand;
+    ga.status = status;
+    ga.zero_counter = nullptr;
+    RowArgs r0;
+    r0.N = N;
+    r0.D = D;
+    r0.K = K;
+    r0.L = L;
+    r0.l = 0;
+    r0.Tc = p.Tc;
+    r0.G = p.Gf;
+    r0.maxs = p.maxs;
+    r0.pair = 0;
+    r0.U = 0;
+    r0.rt0 = 0;
+    r0.nslots = p.NC;
+    r0.cand = cand;
+    r0.rowstat = rowstat;
+    r0.R = R;
+    r0.Rt = Rt;
+    r0.cb = codebooks;
+    r0.stats = level_stats;
+    r0.ids = ids;
+    r0.fb_list = nullptr;  // uncertified rows go to the kernel's exact-scan queue
+    r0.fb_count = fb_count;
+    r0.status = status;
+    r0.last = L == 1;
+    r0.src = features;
+    r0.fb_next = nullptr;
+    r0.offsets = offsets;
+    r0.B = B;
+    FlowArgs fa;
+    fa.L = L;
+    fa.RT = p.RT;
+    fa.NC = p.NC;
+    fa.S = p.S;
+    fa.RPT = p.RPT;
+    fa.NS = p.NS;
+    fa.slice = p.slice;
+    fa.ctr = reinterpret_cast<uint32_t *>(sync);
+    fa.chunk_done = reinterpret_cast<uint32_t *>(sync + 256);
+    fa.cert_done = fa.chunk_done + static_cast<size_t>(L) * p.RT;
+    fa.ex_entry = reinterpret_cast<int4 *>(sync + 256 + align256(2 * static_cast<size_t>(L) * p.RT * 4));
+    fa.ex_part = reinterpret_cast<double2 *>(ws + w.ex_part);
+    fa.fb_level = fb_count;
+    fa.norms = norms;
+    fa.level_stats = level_stats;
+    profile_begin(s);
+    const cudaError_t fe = launch_flow(nch, cb_dtype == RVQ_BF16, f_dtype == RVQ_BF16, p.Gf, s,
+                                       x_is_operand ? tmX : tmA, tmA, tmB3, ga, r0, fa);
+    profile_end(s, L);
+    note_launch();
+    if (fe != cudaSuccess) return RVQ_ERR_CUDA;
+  }
+
   const int64_t row_blocks = (N * 32 + 255) / 256;
   const int fb_blocks = 2 * sms;
   const size_t fb_smem = static_cast<size_t>(D) * sizeof(double);
-  for (int l = 0; l < L; ++l) {
+  for (int l = 0; l < L && !all_levels; ++l) {
     const size_t lvl = static_cast<size_t>(l) * K * D * 2;
     CUtensorMap tmB;
     if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, p.pair ? BN / 2 : BN)) return RVQ_ERR_CUDA;
@@ -1526,6 +2540,8 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ra.maxs = p.maxs;
     ra.pair = p.pair ? 1 : 0;
     ra.U = p.U;
+    ra.rt0 = 0;
+    ra.nslots = 0;
     ra.cand = cand;
     ra.rowstat = rowstat;
     ra.R = R;

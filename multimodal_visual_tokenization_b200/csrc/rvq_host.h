@@ -19,7 +19,7 @@ void note_launch(int n = 1);
 // Profiling of the distance-GEMM launches (see rvq_profile_enable in rvq.h).
 bool profiling_enabled();
 void profile_begin(cudaStream_t s);
-void profile_end(cudaStream_t s);
+void profile_end(cudaStream_t s, int levels = 1);  // levels: RVQ levels the launch covers
 
 inline int check_launch() {
   cudaError_t e = cudaGetLastError();

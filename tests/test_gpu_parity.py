@@ -177,6 +177,62 @@ def test_near_ties_use_exact_rescoring(copies):
         assert fb.sum() > 0
 
 
+@pytest.mark.parametrize("copies", [2, 16])
+def test_near_ties_wide_rows(copies):
+    """The same near-tie groups at D = 1024 (the all-levels kernel): groups of 16 overflow the
+    candidate lists, so their rows take the exact scan split into codeword slices."""
+    rng = np.random.Generator(np.random.PCG64(123 + copies))
+    D, G, N, L = 1024, 16, 300, 2
+    base = rng.standard_normal((G, D)).astype(np.float32)
+    eps = (10.0 ** rng.uniform(-7, -4, size=(copies, G, 1))).astype(np.float32)
+    eps[0] = 0.0
+    lvl0 = (base[None] * (1 + eps)).reshape(copies * G, D)
+    lvl1 = 0.1 * rng.standard_normal((copies * G, D)).astype(np.float32)
+    C = np.stack([lvl0, lvl1])
+    pick = rng.integers(0, G, size=N)
+    x = workloads.round_bf16(base[pick] + 1e-3 * rng.standard_normal((N, D)).astype(np.float32))
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    rep = full_check(x, C, ids, res, rec)
+    print("wide near ties", copies, rep, "fallbacks", fb.tolist())
+    if copies > 8:
+        assert fb[0] > 0
+
+
+def test_exact_queue_overflow_wide_rows():
+    """More uncertifiable rows than the all-levels kernel queues for sliced exact scans: the rest
+    are scanned whole by the warp that found them."""
+    rng = np.random.Generator(np.random.PCG64(131))
+    D, G, copies, N = 1024, 32, 16, 1300
+    base = rng.standard_normal((G, D)).astype(np.float32)
+    eps = (10.0 ** rng.uniform(-7, -5, size=(copies, G, 1))).astype(np.float32)
+    eps[0] = 0.0
+    C = (base[None] * (1 + eps)).reshape(1, copies * G, D)
+    x = workloads.round_bf16(base[rng.integers(0, G, size=N)] + 1e-4 * rng.standard_normal((N, D)).astype(np.float32))
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    full_check(x, C, ids, res, rec)
+    print("queue overflow fallbacks", fb.tolist())
+    assert fb[0] > 1024
+
+
+def test_per_level_path_matches_oracle():
+    """RVQ_PERSISTENT=0 (fresh process): every level as its own GEMM + certificate launches."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, torch, workloads\n"
+        "from tests import parity, test_gpu_parity as t\n"
+        "g = workloads.generate('image', n_override=700)\n"
+        "_, ids, res, rec, fb = t.run_encode(g['x'], g['codebooks'], 'bf16', 'f32')\n"
+        "t.full_check(g['x'], g['codebooks'], ids, res, rec)\n"
+        "print('per-level ok')\n")
+    env = dict(os.environ, RVQ_PERSISTENT="0")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0 and "per-level ok" in out.stdout, out.stdout[-2000:] + out.stderr[-2000:]
+
+
 def test_decode_out_of_range_sets_status():
     C = np.random.Generator(np.random.PCG64(24)).standard_normal((2, 10, 64)).astype(np.float32)
     tok = mvt.Tokenizer(dev(C, "f32"))
