@@ -36,7 +36,7 @@ METRIC = "RVQ encode Mtokens/s (L levels, K codes, dim D) and % tensor-core peak
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 512 << 20          # > 126 MB L2
 GEMM_KERNEL_SRC = os.path.join(ROOT, "multimodal_visual_tokenization_b200", "csrc", "rvq_encode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dist_topk_traffic.txt")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "encode_traffic.txt")
 
 
 def parse_args(argv=None):
@@ -138,17 +138,19 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def read_traffic(workload):
-    """ncu DRAM bytes per distance-GEMM launch for this workload, if captured from the current
-    kernel source (profiles/dist_topk_traffic.txt lines: workload bytes_per_launch source_sha)."""
+def read_traffic(workload, kernel):
+    """ncu DRAM bytes per launch of the dominant encode kernel for this workload, if captured from
+    the current kernel source (profiles/encode_traffic.txt lines: workload kernel bytes_per_launch
+    source_sha)."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     sha = file_sha(GEMM_KERNEL_SRC)
     with open(TRAFFIC_FILE) as f:
         for ln in f:
             parts = ln.split()
-            if len(parts) >= 3 and not ln.startswith("#") and parts[0] == workload and parts[2] == sha:
-                return float(parts[1])
+            if (len(parts) >= 4 and not ln.startswith("#") and parts[0] == workload and parts[1] == kernel
+                    and parts[3] == sha):
+                return float(parts[2])
     return None
 
 
@@ -405,14 +407,20 @@ def run_ours(args, rank, world, local_rank):
     long_step = ms_per_step > 20.0
     peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
     peak = float(peaks.get(peak_key, PEAKS_FALLBACK[peak_key]))
-    flops_per_launch = 2.0 * N * K * D  # one level: every (row, codeword) dot product
-    gemm_avg_ms = gemm_ms / max(1, gemm_n)
-    achieved = flops_per_launch / (gemm_avg_ms / 1e3) / 1e12
-    traffic = read_traffic(args.workload)
+    # the dominant encode kernel: one launch per level (distance GEMM + top-8), or one launch for
+    # all levels (dataflow kernel: GEMM, top-8, certificate and residual update)
+    code, lpl = mvt.rvq_encode_levels_per_launch(N, D, L, K)
+    check(code, "levels per launch")
+    kernel = "encode_flow_kernel" if lpl > 1 else "dist_topk_kernel"
+    flops_per_launch = 2.0 * N * K * D * lpl  # every (row, codeword) dot product of the levels covered
+    launches = max(1, gemm_n // lpl)
+    launch_ms = gemm_ms / launches
+    achieved = flops_per_launch / (launch_ms / 1e3) / 1e12
+    traffic = read_traffic(args.workload, kernel)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "dist_topk_kernel", "launch_ms": gemm_avg_ms,
-                "launches_timed": gemm_n, "flops_per_launch": flops_per_launch,
+                "kernel": kernel, "levels_per_launch": lpl, "launch_ms": launch_ms,
+                "launches_timed": launches, "flops_per_launch": flops_per_launch,
                 "peak_source": f"{peak_src} {peak_key}"}
 
     # -------------------------------------------------- quick parity sample + CPU baseline

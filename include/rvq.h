@@ -166,13 +166,18 @@ RVQ_API const char *rvq_status_str(int status);
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on
  *   its stream (not for use inside stream capture); rvq_profile_enable(0) stops and clears.
  * rvq_profile_read: synchronises on the recorded events and returns the number of RVQ levels the
- *   bracketed launches covered (a per-level distance-GEMM launch counts 1; the all-levels persistent
- *   encode kernel, which also runs the certificate phases, counts L) and their summed device time
+ *   bracketed launches covered (a per-level distance-GEMM launch counts 1; the all-levels dataflow
+ *   encode kernel, which also runs the certificate work, counts L) and their summed device time
  *   in milliseconds since the last enable.
+ * rvq_encode_levels_per_launch: for an encode of this shape on the current device, the number of
+ *   RVQ levels one bracketed launch covers (L when the all-levels kernel runs, else 1), so that a
+ *   profiler can turn rvq_profile_read's totals into per-launch figures.  Same argument checks as
+ *   rvq_encode_workspace_size.
  */
 RVQ_API int64_t rvq_launch_count(void);
 RVQ_API int rvq_profile_enable(int enable);
 RVQ_API int rvq_profile_read(int64_t *gemm_launches, double *gemm_ms);
+RVQ_API int rvq_encode_levels_per_launch(int64_t N, int D, int L, int K, int *levels);
 
 #ifdef __cplusplus
 }

@@ -1836,8 +1836,10 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
       int64_t claimed = -1;
       int en = 0, el = 0;
       if (lane == 0) {
-        const uint32_t s = ld_acquire_gpu(ex_next);
-        const uint32_t rows = min(ld_acquire_gpu(ex_rows), static_cast<uint32_t>(EXACT_QCAP));
+        // plain (relaxed) polling reads; the entry's ready flag is acquired before it is used
+        const uint32_t rows = min(*reinterpret_cast<const volatile uint32_t *>(ex_rows),
+                                  static_cast<uint32_t>(EXACT_QCAP));
+        const uint32_t s = rows ? *reinterpret_cast<const volatile uint32_t *>(ex_next) : 0u;
         if (s < rows * static_cast<uint32_t>(fa.NS)) {
           const int q = static_cast<int>(s / fa.NS);
           if (ld_acquire_gpu(reinterpret_cast<const uint32_t *>(&fa.ex_entry[q].z)) != 0 &&
@@ -1919,17 +1921,16 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
       }
       return true;
     };
-    // Wait for *ctr >= target, running exact-scan slices meanwhile.
+    // Wait for *ctr >= target, running exact-scan slices meanwhile.  Each poll reads the
+    // (per row tile) counter and, unless the exact-scan queue is empty, its head; the progress
+    // word for the time limit is read every 16th poll.
     auto wait_helping = [&](const uint32_t *ctr, uint32_t target) -> bool {
       uint32_t last_p = 0;
       uint64_t t0 = 0;
       bool first = true;
-      while (true) {
-        uint32_t c = 0, pr = 0;
-        if (lane == 0) {
-          c = ld_acquire_gpu(ctr);
-          pr = *reinterpret_cast<const volatile uint32_t *>(progress);
-        }
+      for (uint32_t iter = 0;; ++iter) {
+        uint32_t c = 0;
+        if (lane == 0) c = ld_acquire_gpu(ctr);
         c = __shfl_sync(0xffffffffu, c, 0);
         if (c >= target) return true;
         if (*abort_flag) return false;
@@ -1937,17 +1938,21 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
           first = true;
           continue;
         }
-        pr = __shfl_sync(0xffffffffu, pr, 0);
-        const uint64_t now = global_timer_ns();
-        if (first || pr != last_p) {
-          first = false;
-          last_p = pr;
-          t0 = now;
-        } else if (now - t0 > 2000000000ull) {
-          *abort_flag = 1;
-          return false;
+        if (first || (iter & 15) == 0) {
+          uint32_t pr = 0;
+          if (lane == 0) pr = *reinterpret_cast<const volatile uint32_t *>(progress);
+          pr = __shfl_sync(0xffffffffu, pr, 0);
+          const uint64_t now = global_timer_ns();
+          if (first || pr != last_p) {
+            first = false;
+            last_p = pr;
+            t0 = now;
+          } else if (now - t0 > 2000000000ull) {
+            *abort_flag = 1;
+            return false;
+          }
         }
-        __nanosleep(200);
+        __nanosleep(500);
       }
     };
 
@@ -2063,6 +2068,16 @@ inline bool persistent_enabled() {
   return v != 0;
 }
 
+// RVQ_FLOW_NC=n (1..16) fixes the chunks per row tile of the all-levels kernel (tuning knob).
+inline int flow_chunks_forced() {
+  static int v = [] {
+    const char *e = getenv("RVQ_FLOW_NC");
+    const int n = e ? atoi(e) : 0;
+    return n >= 1 && n <= MAX_SLOTS ? n : 0;
+  }();
+  return v;
+}
+
 // Row chunks (float4 per lane) of the register-resident row kernels for feature width D <= 1024.
 inline int row_chunks(int D) { return D <= 128 ? 1 : D <= 256 ? 2 : D <= 512 ? 4 : 8; }
 
@@ -2120,6 +2135,7 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
     p.Gf = sms0;
     // enough chunks per level to keep every CTA busy and finish a row tile soon after it starts
     int nc = static_cast<int>(std::min<int64_t>(MAX_SLOTS, std::max<int64_t>(1, (4 * p.Gf + p.RT - 1) / p.RT)));
+    if (flow_chunks_forced() > 0) nc = flow_chunks_forced();
     nc = std::min(nc, p.Tc);
     p.S = (p.Tc + nc - 1) / nc;
     p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
@@ -2362,6 +2378,18 @@ extern "C" int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t 
   if (st != RVQ_OK) return st;
   const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, L, sms);
   *bytes = enc::make_layout(N, D, p).total;
+  return RVQ_OK;
+}
+
+extern "C" int rvq_encode_levels_per_launch(int64_t N, int D, int L, int K, int *levels) {
+  using namespace rvq;
+  if (!levels || N < 0 || D < 1 || L < 1 || K < 1) return RVQ_ERR_ARG;
+  if (L > 64 || D < 64 || D > 4096 || D % 64 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  int sms = 0;
+  int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, L, sms);
+  *levels = p.flow ? L : 1;
   return RVQ_OK;
 }
 

@@ -71,6 +71,10 @@ def test_host_argument_checks(lib):
     assert enc(*no_ws) == -3
     mis = list(args); mis[2] = 5; mis[0] = 18
     assert enc(*mis) == -1                                                   # misaligned features
+    lv = ctypes.c_int32(0)
+    assert L.rvq_encode_levels_per_launch(100, 1024, 4, 8192, None) == -1    # no output
+    assert L.rvq_encode_levels_per_launch(100, 1000, 4, 8192, ctypes.byref(lv)) == -2   # D % 64
+    assert L.rvq_encode_levels_per_launch(100, 1024, 65, 8192, ctypes.byref(lv)) == -2  # L > 64
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -298,6 +298,22 @@ def test_launch_count_and_profile_hooks():
     assert mvt.rvq_launch_count() - before == 1 + 3 * g["spec"].L
 
 
+def test_levels_per_launch_query():
+    """D in (512, 1024] runs all levels in one launch; other widths launch per level."""
+    assert mvt.rvq_encode_levels_per_launch(4096, 1024, 4, 8192) == (0, 4)
+    assert mvt.rvq_encode_levels_per_launch(4096, 768, 3, 1000) == (0, 3)
+    assert mvt.rvq_encode_levels_per_launch(4096, 256, 4, 8192) == (0, 1)
+    assert mvt.rvq_encode_levels_per_launch(4096, 2048, 4, 8192) == (0, 1)
+    g = workloads.generate("image", n_override=300)
+    tok = mvt.Tokenizer(dev(g["codebooks"], "f32"))
+    x = dev(g["x"], "bf16")
+    assert mvt.rvq_profile_enable(True) == 0
+    tok.encode(x)
+    code, n, ms = mvt.rvq_profile_read()
+    mvt.rvq_profile_enable(False)
+    assert code == 0 and n == g["spec"].L and ms > 0
+
+
 def test_wide_features_use_streaming_rows():
     """D > 1024 takes the path that materialises the fp32 residual and streams rows."""
     rng = np.random.Generator(np.random.PCG64(27))
