@@ -413,14 +413,14 @@ def run_ours(args, rank, world, local_rank):
     check(code, "levels per launch")
     kernel = "encode_flow_kernel" if lpl > 1 else "dist_topk_kernel"
     flops_per_launch = 2.0 * N * K * D * lpl  # every (row, codeword) dot product of the levels covered
-    launches = max(1, gemm_n // lpl)
-    launch_ms = gemm_ms / launches
+    enc_launches = max(1, gemm_n // lpl)
+    launch_ms = gemm_ms / enc_launches
     achieved = flops_per_launch / (launch_ms / 1e3) / 1e12
     traffic = read_traffic(args.workload, kernel)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": kernel, "levels_per_launch": lpl, "launch_ms": launch_ms,
-                "launches_timed": launches, "flops_per_launch": flops_per_launch,
+                "launches_timed": enc_launches, "flops_per_launch": flops_per_launch,
                 "peak_source": f"{peak_src} {peak_key}"}
 
     # -------------------------------------------------- quick parity sample + CPU baseline

@@ -1298,9 +1298,9 @@ inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blo
 // so level l+1 of a row tile starts while later row tiles of level l are still being scored,
 // and the certificate work runs under the tensor-core work.  Every wait is bounded: it gives up
 // when neither its counter nor the grid's progress word has moved for two seconds.
-// Certificate warps of the all-levels kernel for D in (512, 1024], next to 8 epilogue warps:
-// they fill the block up to 16 warps (the register budget per thread is set by the warp count
-// rounded up to a multiple of four).
+// Certificate warps of the all-levels kernel, next to 8 epilogue warps: they fill the block up
+// to 16 warps (the register budget per thread is set by the warp count rounded up to a multiple
+// of four).
 constexpr int FLOW_RW_WIDE = 5;
 constexpr int EXACT_QCAP = 1024;   // queued rows whose exact scan is split into slices
 constexpr int EXACT_NS_MAX = 256;  // codeword slices per queued row
@@ -2126,9 +2126,9 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
 
   const int nch = row_chunks(D);
   p.L = L;
-  // D in (512, 1024] only: at D <= 256 the distance epilogue is issue-bound and leaves the block
-  // room for one certificate warp, which cannot keep up (measured), so levels run one by one
-  p.flow = !p.pair && D <= 1024 && nch == 8 && persistent_enabled() &&
+  // D in (128, 256] and (512, 1024]: 8 epilogue + 5 certificate warps (other widths run the
+  // levels one by one)
+  p.flow = !p.pair && D <= 1024 && (nch == 2 || nch == 8) && persistent_enabled() &&
            static_cast<uint64_t>(N) * static_cast<uint64_t>(L) < (uint64_t(1) << 32);
   p.NC = p.S = p.RPT = p.NS = p.slice = p.Gf = 0;
   if (p.flow) {
@@ -2233,9 +2233,9 @@ inline bool set_gemm_attr() {
                               GemmCfg<EPI, PAIR>::SMEM) == cudaSuccess;
 }
 
-// Epilogue warps of the distance GEMM.  A short feature width gives little MMA time per tile to
-// hide the epilogue behind, so more warps share it (measured: 16 warps win at D <= 256, 8 above).
-// RVQ_EPI_WARPS=4|8|16 overrides the choice (tuning knob).
+// Epilogue warps of the distance GEMM: 8 (measured with the bit-mask insert path: 8 beat 16 at
+// D = 256, 31.4 vs 35.0 ms per offline level).  RVQ_EPI_WARPS=4|8|16 overrides the choice
+// (tuning knob).
 inline int epilogue_warps(int D) {
   static int forced = [] {
     const char *e = getenv("RVQ_EPI_WARPS");
@@ -2243,7 +2243,8 @@ inline int epilogue_warps(int D) {
     return (v == 4 || v == 8 || v == 16) ? v : 0;
   }();
   if (forced) return forced;
-  return D <= 256 ? 16 : 8;
+  (void)D;
+  return 8;
 }
 
 inline bool gemm_attrs_ready(int epi) {
@@ -2308,7 +2309,8 @@ inline int resident_pair_clusters(int D) {
   return epi == 4 ? max_pair_clusters<4>() : epi == 16 ? max_pair_clusters<16>() : max_pair_clusters<8>();
 }
 
-// All-levels dataflow encode, instantiated for D in (512, 1024] (see FLOW_RW_WIDE).
+// All-levels dataflow encode, instantiated for 2 (D in (128, 256]) and 8 (D in (512, 1024])
+// float4 row chunks.
 
 template <int EPI, int RW, bool CB, bool XB, int NCH>
 inline bool set_flow_attr() {
@@ -2322,7 +2324,9 @@ inline bool flow_attrs_ready() {
   std::call_once(once, [] {
     constexpr int RWD = FLOW_RW_WIDE;
     ok = set_flow_attr<8, RWD, false, false, 8>() && set_flow_attr<8, RWD, false, true, 8>() &&
-         set_flow_attr<8, RWD, true, false, 8>() && set_flow_attr<8, RWD, true, true, 8>();
+         set_flow_attr<8, RWD, true, false, 8>() && set_flow_attr<8, RWD, true, true, 8>() &&
+         set_flow_attr<8, RWD, false, false, 2>() && set_flow_attr<8, RWD, false, true, 2>() &&
+         set_flow_attr<8, RWD, true, false, 2>() && set_flow_attr<8, RWD, true, true, 2>();
   });
   return ok;
 }
@@ -2347,6 +2351,12 @@ inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cud
                                const CUtensorMap &tmA, const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra,
                                const FlowArgs &fa) {
   constexpr int RWD = FLOW_RW_WIDE;
+  if (nch == 2) {
+    if (cb_bf16) return x_bf16 ? launch_flow_t<8, RWD, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                               : launch_flow_t<8, RWD, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    return x_bf16 ? launch_flow_t<8, RWD, false, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                  : launch_flow_t<8, RWD, false, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  }
   if (nch != 8) return cudaErrorInvalidValue;
   if (cb_bf16) return x_bf16 ? launch_flow_t<8, RWD, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
                              : launch_flow_t<8, RWD, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);

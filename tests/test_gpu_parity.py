@@ -299,10 +299,12 @@ def test_launch_count_and_profile_hooks():
 
 
 def test_levels_per_launch_query():
-    """D in (512, 1024] runs all levels in one launch; other widths launch per level."""
+    """D in (128, 256] or (512, 1024] runs all levels in one launch; other widths launch per level."""
     assert mvt.rvq_encode_levels_per_launch(4096, 1024, 4, 8192) == (0, 4)
     assert mvt.rvq_encode_levels_per_launch(4096, 768, 3, 1000) == (0, 3)
-    assert mvt.rvq_encode_levels_per_launch(4096, 256, 4, 8192) == (0, 1)
+    assert mvt.rvq_encode_levels_per_launch(4096, 256, 4, 8192) == (0, 4)
+    assert mvt.rvq_encode_levels_per_launch(4096, 128, 4, 8192) == (0, 1)
+    assert mvt.rvq_encode_levels_per_launch(4096, 512, 4, 8192) == (0, 1)
     assert mvt.rvq_encode_levels_per_launch(4096, 2048, 4, 8192) == (0, 1)
     g = workloads.generate("image", n_override=300)
     tok = mvt.Tokenizer(dev(g["codebooks"], "f32"))
