@@ -179,6 +179,18 @@ RVQ_API int rvq_profile_enable(int enable);
 RVQ_API int rvq_profile_read(int64_t *gemm_launches, double *gemm_ms);
 RVQ_API int rvq_encode_levels_per_launch(int64_t N, int D, int L, int K, int *levels);
 
+/*
+ * Self-test of the bounded waits (no counterpart on the pages).  Every spin of the encode kernels
+ * (an mbarrier phase, a grid-wide counter) gives up after a time limit and reports
+ * RVQ_ERR_TIMEOUT through the status word instead of hanging the GPU.  This call launches one
+ * block that waits on an mbarrier phase nothing completes and on *counter, which the caller keeps
+ * at 0, each for at most limit_us microseconds (1 .. 10^7), and then writes RVQ_ERR_TIMEOUT into
+ * *status (device int32, first error wins) when both waits gave up as designed, RVQ_ERR_ARG
+ * otherwise.  counter and status are caller-owned device pointers.  Returns RVQ_OK when the
+ * launch was enqueued, RVQ_ERR_ARG for bad arguments.
+ */
+RVQ_API int rvq_selftest_wait_timeout(const uint32_t *counter, int32_t *status, int64_t limit_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

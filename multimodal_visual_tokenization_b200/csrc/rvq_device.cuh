@@ -133,6 +133,33 @@ __device__ __forceinline__ void red_release_add_gpu(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Wait until *ctr >= target (acquire).  Gives up, sets *abort and returns false when neither
+// *ctr nor the grid's progress word has moved for limit_ns.
+static __device__ __noinline__ bool wait_count(const uint32_t *ctr, uint32_t target, const uint32_t *progress,
+                                               volatile int *abort, uint64_t limit_ns = 2000000000ull) {
+  uint32_t c = ld_acquire_gpu(ctr);
+  if (c >= target) return true;
+  uint32_t last_c = c;
+  uint32_t last_p = *reinterpret_cast<const volatile uint32_t *>(progress);
+  uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(100);
+    c = ld_acquire_gpu(ctr);
+    if (c >= target) return true;
+    if (*abort) return false;
+    const uint32_t pr = *reinterpret_cast<const volatile uint32_t *>(progress);
+    const uint64_t now = global_timer_ns();
+    if (c != last_c || pr != last_p) {
+      last_c = c;
+      last_p = pr;
+      t0 = now;
+    } else if (now - t0 > limit_ns) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16),
 // completion counted on `bar` in bytes.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

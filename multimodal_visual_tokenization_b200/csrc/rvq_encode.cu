@@ -1298,10 +1298,15 @@ inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blo
 // so level l+1 of a row tile starts while later row tiles of level l are still being scored,
 // and the certificate work runs under the tensor-core work.  Every wait is bounded: it gives up
 // when neither its counter nor the grid's progress word has moved for two seconds.
-// Certificate warps of the all-levels kernel, next to 8 epilogue warps: they fill the block up
-// to 16 warps (the register budget per thread is set by the warp count rounded up to a multiple
-// of four).
+// Epilogue and certificate warps of the all-levels kernel.  With the three GEMM-role warps they
+// fill the block to 16 warps (the register budget per thread is set by the warp count rounded up
+// to a multiple of four).  8 + 5 at both widths: at D = 1024, 4 epilogue + 9 certificate warps
+// measured 9% slower on image (the epilogue then shares its SM sub-partition with more
+// certificate work), although 4 epilogue warps are faster in the per-level kernel.
+constexpr int FLOW_EPI_WIDE = 8;
 constexpr int FLOW_RW_WIDE = 5;
+constexpr int FLOW_EPI_NARROW = 8;
+constexpr int FLOW_RW_NARROW = 5;
 constexpr int EXACT_QCAP = 1024;   // queued rows whose exact scan is split into slices
 constexpr int EXACT_NS_MAX = 256;  // codeword slices per queued row
 
@@ -1320,33 +1325,6 @@ struct FlowArgs {
   const float *norms;    // [L, K]
   const float *level_stats;
 };
-
-// Wait until *ctr >= target (acquire).  Gives up, sets *abort and returns false when neither
-// *ctr nor the grid's progress word has moved for limit_ns.
-__device__ __noinline__ bool wait_count(const uint32_t *ctr, uint32_t target, const uint32_t *progress,
-                                        volatile int *abort, uint64_t limit_ns = 2000000000ull) {
-  uint32_t c = ld_acquire_gpu(ctr);
-  if (c >= target) return true;
-  uint32_t last_c = c;
-  uint32_t last_p = *reinterpret_cast<const volatile uint32_t *>(progress);
-  uint64_t t0 = global_timer_ns();
-  while (true) {
-    __nanosleep(100);
-    c = ld_acquire_gpu(ctr);
-    if (c >= target) return true;
-    if (*abort) return false;
-    const uint32_t pr = *reinterpret_cast<const volatile uint32_t *>(progress);
-    const uint64_t now = global_timer_ns();
-    if (c != last_c || pr != last_p) {
-      last_c = c;
-      last_p = pr;
-      t0 = now;
-    } else if (now - t0 > limit_ns) {
-      *abort = 1;
-      return false;
-    }
-  }
-}
 
 // Publish this warp's global writes and add v (warp-uniform) to *ctr.  TMA: the writes are also
 // made visible to the async proxy (later TMA loads of the residual operand).
@@ -2141,7 +2119,7 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
     p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
     p.maxs = std::max(p.maxs, p.NC);
     // certificate tasks: about two per certificate warp per level, at most one row tile each
-    const int64_t cw = static_cast<int64_t>(p.Gf) * FLOW_RW_WIDE;
+    const int64_t cw = static_cast<int64_t>(p.Gf) * (nch == 8 ? FLOW_RW_WIDE : FLOW_RW_NARROW);
     int tg = 1;
     while (tg < 64 && static_cast<int64_t>(tg) * p.RT < 2 * cw) tg *= 2;
     p.RPT = BM / tg;
@@ -2233,9 +2211,9 @@ inline bool set_gemm_attr() {
                               GemmCfg<EPI, PAIR>::SMEM) == cudaSuccess;
 }
 
-// Epilogue warps of the distance GEMM: 8 (measured with the bit-mask insert path: 8 beat 16 at
-// D = 256, 31.4 vs 35.0 ms per offline level).  RVQ_EPI_WARPS=4|8|16 overrides the choice
-// (tuning knob).
+// Epilogue warps of the per-level distance GEMM: 4 above D = 512 (a tile's longer MMA hides a
+// 4-warp epilogue: 5% faster than 8 at D = 1024), else 8 (8 beat 16 at D = 256: 31.4 vs 35.0 ms
+// per offline level, and 4: 33.2 ms).  RVQ_EPI_WARPS=4|8|16 overrides the choice (tuning knob).
 inline int epilogue_warps(int D) {
   static int forced = [] {
     const char *e = getenv("RVQ_EPI_WARPS");
@@ -2243,8 +2221,7 @@ inline int epilogue_warps(int D) {
     return (v == 4 || v == 8 || v == 16) ? v : 0;
   }();
   if (forced) return forced;
-  (void)D;
-  return 8;
+  return D > 512 ? 4 : 8;
 }
 
 inline bool gemm_attrs_ready(int epi) {
@@ -2322,11 +2299,11 @@ inline bool flow_attrs_ready() {
   static std::once_flag once;
   static bool ok = false;
   std::call_once(once, [] {
-    constexpr int RWD = FLOW_RW_WIDE;
-    ok = set_flow_attr<8, RWD, false, false, 8>() && set_flow_attr<8, RWD, false, true, 8>() &&
-         set_flow_attr<8, RWD, true, false, 8>() && set_flow_attr<8, RWD, true, true, 8>() &&
-         set_flow_attr<8, RWD, false, false, 2>() && set_flow_attr<8, RWD, false, true, 2>() &&
-         set_flow_attr<8, RWD, true, false, 2>() && set_flow_attr<8, RWD, true, true, 2>();
+    constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW;
+    ok = set_flow_attr<EW, RWD, false, false, 8>() && set_flow_attr<EW, RWD, false, true, 8>() &&
+         set_flow_attr<EW, RWD, true, false, 8>() && set_flow_attr<EW, RWD, true, true, 8>() &&
+         set_flow_attr<EN, RN, false, false, 2>() && set_flow_attr<EN, RN, false, true, 2>() &&
+         set_flow_attr<EN, RN, true, false, 2>() && set_flow_attr<EN, RN, true, true, 2>();
   });
   return ok;
 }
@@ -2350,18 +2327,18 @@ inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tm
 inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cudaStream_t s, const CUtensorMap &tmA0,
                                const CUtensorMap &tmA, const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra,
                                const FlowArgs &fa) {
-  constexpr int RWD = FLOW_RW_WIDE;
+  constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW;
   if (nch == 2) {
-    if (cb_bf16) return x_bf16 ? launch_flow_t<8, RWD, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                               : launch_flow_t<8, RWD, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
-    return x_bf16 ? launch_flow_t<8, RWD, false, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                  : launch_flow_t<8, RWD, false, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    if (cb_bf16) return x_bf16 ? launch_flow_t<EN, RN, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                               : launch_flow_t<EN, RN, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    return x_bf16 ? launch_flow_t<EN, RN, false, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                  : launch_flow_t<EN, RN, false, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
   }
   if (nch != 8) return cudaErrorInvalidValue;
-  if (cb_bf16) return x_bf16 ? launch_flow_t<8, RWD, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                             : launch_flow_t<8, RWD, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
-  return x_bf16 ? launch_flow_t<8, RWD, false, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                : launch_flow_t<8, RWD, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  if (cb_bf16) return x_bf16 ? launch_flow_t<EW, RWD, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                             : launch_flow_t<EW, RWD, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  return x_bf16 ? launch_flow_t<EW, RWD, false, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                : launch_flow_t<EW, RWD, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
 }
 
 inline cudaError_t launch_gemm(int epi, bool pair, int groups, cudaStream_t s, const CUtensorMap &tmA,

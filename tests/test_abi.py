@@ -75,6 +75,8 @@ def test_host_argument_checks(lib):
     assert L.rvq_encode_levels_per_launch(100, 1024, 4, 8192, None) == -1    # no output
     assert L.rvq_encode_levels_per_launch(100, 1000, 4, 8192, ctypes.byref(lv)) == -2   # D % 64
     assert L.rvq_encode_levels_per_launch(100, 1024, 65, 8192, ctypes.byref(lv)) == -2  # L > 64
+    assert L.rvq_selftest_wait_timeout(None, 16, 1000, None) == -1               # no counter
+    assert L.rvq_selftest_wait_timeout(16, 16, 0, None) == -1                  # limit out of range
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -113,6 +113,10 @@ def test_detok_decode_and_round_trip():
 EDGE = [
     # N, D, L, K, f_dtype, cb_dtype
     (1, 64, 2, 16, "f32", "f32"),
+    (1000, 256, 3, 700, "f32", "f32"),      # all-levels kernel: fp32 features, ragged N and K
+    (300, 1024, 1, 300, "f32", "f32"),      # all-levels kernel, one level
+    (129, 1024, 3, 257, "bf16", "bf16"),    # all-levels kernel, two row tiles
+    (2, 256, 4, 5000, "bf16", "f32"),       # all-levels kernel, one row tile
     (127, 64, 3, 300, "f32", "f32"),
     (129, 128, 2, 257, "bf16", "f32"),
     (300, 256, 2, 1, "f32", "f32"),
@@ -257,6 +261,38 @@ def test_bad_offsets_set_status():
     tok.encode(dev(x, "f32"), offsets=off, status=st, check=False)
     torch.cuda.synchronize()
     assert int(st.item()) == -1
+
+
+def test_bad_offsets_set_status_all_levels_kernel():
+    """The all-levels kernel checks the packed-batch offsets too (D = 1024)."""
+    rng = np.random.Generator(np.random.PCG64(125))
+    C = rng.standard_normal((2, 300, 1024)).astype(np.float32)
+    x = rng.standard_normal((200, 1024)).astype(np.float32)
+    tok = mvt.Tokenizer(dev(C, "f32"))
+    assert mvt.rvq_encode_levels_per_launch(200, 1024, 2, 300) == (0, 2)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    off = torch.tensor([0, 120, 90, 200], dtype=torch.int64, device="cuda")
+    tok.encode(dev(x, "f32"), offsets=off, status=st, check=False)
+    torch.cuda.synchronize()
+    assert int(st.item()) == -1
+
+
+def test_bounded_waits_give_up():
+    """A wait on an mbarrier phase and on a counter that nothing completes ends after its limit
+    with RVQ_ERR_TIMEOUT in the status word, and the context stays usable."""
+    import time
+    ctr = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    assert mvt.rvq_selftest_wait_timeout(ctr, st, 50_000) == 0
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert int(st.item()) == -6, mvt.rvq_status_str(int(st.item()))
+    assert 0.045 < dt < 5.0, dt
+    g = workloads.generate("tiny")
+    _, ids, res, rec, fb = run_encode(g["x"], g["codebooks"])
+    full_check(g["x"], g["codebooks"], ids, res, rec)
 
 
 def test_empty_batch_is_noop():
