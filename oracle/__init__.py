@@ -63,6 +63,7 @@ def _declare(lib):
                                           f64p, i32p, f64p, f64p, I]
     lib.rvq_oracle_distances.argtypes = [f64p, f32p, I, I, f64p]
     lib.rvq_oracle_max_threads.argtypes = [I]
+    lib.rvq_oracle_embed_backward.argtypes = [i32p, I64, I, I, I, f32p, f64p, i64p, f64p, I]
     for fn in ("rvq_oracle_encode", "rvq_oracle_decode", "rvq_oracle_check_path",
                "rvq_oracle_distances", "rvq_oracle_max_threads"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -155,3 +156,24 @@ def distances(r, C_l, lib=None):
     if rc != 0:
         raise OracleError(rc)
     return out
+
+
+def embed_backward(ids, g, K, bounds: bool = False, threads: int = 0, lib=None):
+    """grad [L,K,H] fp64 of e[n] = sum_l E_l[ids[n,l]] given g = dLoss/de [N,H] (rows summed in
+    ascending n); with bounds=True also count [L,K] and absum [L,K,H] (sum of |g| per row)."""
+    lib = lib or load()
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    g = _f32(g)
+    N, L = ids.shape
+    N2, H = g.shape
+    assert N == N2
+    grad = np.zeros((L, K, H), np.float64)
+    count = np.zeros((L, K), np.int64) if bounds else None
+    absum = np.zeros((L, K, H), np.float64) if bounds else None
+    rc = lib.rvq_oracle_embed_backward(_p(ids, ctypes.c_int32), N, L, K, H, _p(g, ctypes.c_float),
+                                       _p(grad, ctypes.c_double),
+                                       _p(count, ctypes.c_int64) if bounds else None,
+                                       _p(absum, ctypes.c_double) if bounds else None, int(threads))
+    if rc != 0:
+        raise OracleError(rc)
+    return (grad, count, absum) if bounds else grad

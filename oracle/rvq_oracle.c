@@ -243,3 +243,43 @@ int rvq_oracle_distances(const double *r, const float *C_l, int K, int D, double
     for (int k = 0; k < K; ++k) d[k] = sq_dist(r, C_l + (size_t)k * D, D);
     return ORACLE_OK;
 }
+
+/*
+ * Gradient of the visual-token embedding of the backbone (LongCat-2.5 technical blog,
+ * "Visual Primitive Modeling": the visual codebook embeddings are learned jointly with the
+ * backbone).  The embedding of a token is the same gather-sum as decode, with learned tables E:
+ *     e[n] = sum_l E_l[ids[n,l]]
+ * so its gradient with respect to the tables, given g = dLoss/de [N,H], is
+ *     grad[l, k, :] = sum over n with ids[n,l] == k of g[n, :]
+ * accumulated here in fp64, in ascending n, into the caller's array (zero it for a fresh
+ * gradient).  count[l,k] (optional) receives the number of such n, absum[l,k,:] (optional) the
+ * sum of |g[n,:]| over them: the magnitudes that bound the rounding of an fp32 sum of the same
+ * terms taken in any order.  An id outside [0, K) returns ORACLE_ERR_ID_RANGE and adds nothing.
+ * Parallel over levels only, so every (l, k) row is summed by one thread in row order.
+ */
+int rvq_oracle_embed_backward(const int32_t *ids, int64_t N, int L, int K, int H, const float *g,
+                              double *grad, int64_t *count, double *absum, int nthreads)
+{
+    if (!ids || !g || !grad || H <= 0 || L <= 0 || K <= 0 || N < 0) return ORACLE_ERR_ARG;
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int l = 0; l < L; ++l) {
+        for (int64_t n = 0; n < N; ++n) {
+            int32_t id = ids[(size_t)n * L + l];
+            if (id < 0 || id >= K) {
+                bad = 1;
+                continue;
+            }
+            double *dst = grad + ((size_t)l * K + (size_t)id) * H;
+            const float *src = g + (size_t)n * H;
+            for (int i = 0; i < H; ++i) dst[i] = dst[i] + (double)src[i];
+            if (count) count[(size_t)l * K + (size_t)id] += 1;
+            if (absum) {
+                double *a = absum + ((size_t)l * K + (size_t)id) * H;
+                for (int i = 0; i < H; ++i) a[i] = a[i] + fabs((double)src[i]);
+            }
+        }
+    }
+    return bad ? ORACLE_ERR_ID_RANGE : ORACLE_OK;
+}

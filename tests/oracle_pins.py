@@ -10,7 +10,13 @@ disagrees with:
     margin; integer-valued decode),
   * invariants (recon + residual == x; residual norms never grow when every level
     holds a zero codeword; exact ties go to the lowest index),
-  * the hand-worked example in tests/golden/rvq_toy_2d.txt.
+  * the hand-worked example in tests/golden/rvq_toy_2d.txt,
+and the gradient of the embedding e[n] = sum_l E_l[ids[n,l]] (the decode gather-sum with
+learned tables) with:
+  * the adjoint identity <decode(ids, E), G> = <E, backward(ids, G)> (decode pinned above),
+  * a permutation of ids per level (each gradient row is one input row, exactly),
+  * numpy's unbuffered scatter-add (np.add.at) on small inputs,
+  * column sums (every input row lands in exactly one row per level) and the magnitude bounds.
 """
 from __future__ import annotations
 
@@ -231,6 +237,61 @@ def pin_check_path(lib):
                        rtol=1e-13)
 
 
+def _embed_case(seed, N, L, K, H, skew=False):
+    rng = _rng(seed)
+    if skew:  # a few very popular ids, as with Zipf-distributed level-0 tokens
+        ids = np.minimum(rng.zipf(1.3, size=(N, L)) - 1, K - 1).astype(np.int32)
+    else:
+        ids = rng.integers(0, K, size=(N, L)).astype(np.int32)
+    g = rng.standard_normal((N, H)).astype(np.float32)
+    return ids, g
+
+
+def pin_embed_adjoint(lib):
+    for seed, (N, L, K, H, skew) in enumerate([(300, 3, 17, 24, False), (500, 2, 64, 8, True),
+                                               (40, 5, 3, 16, False)]):
+        ids, g = _embed_case(900 + seed, N, L, K, H, skew)
+        E = _rng(950 + seed).standard_normal((L, K, H)).astype(np.float32)
+        e = oracle.decode(ids, E, lib=lib)                       # forward (pinned separately)
+        grad = oracle.embed_backward(ids, g, K, lib=lib)
+        lhs = float(np.sum(e * g.astype(np.float64)))
+        rhs = float(np.sum(E.astype(np.float64) * grad))
+        assert abs(lhs - rhs) <= 1e-11 * (abs(lhs) + abs(rhs) + 1.0), (lhs, rhs)
+
+
+def pin_embed_permutation(lib):
+    rng = _rng(960)
+    L, K, H = 3, 50, 12
+    ids = np.stack([rng.permutation(K) for _ in range(L)], axis=1).astype(np.int32)  # N = K
+    g = rng.standard_normal((K, H)).astype(np.float32)
+    grad = oracle.embed_backward(ids, g, K, lib=lib)
+    for l in range(L):
+        assert np.array_equal(grad[l, ids[:, l]], g.astype(np.float64))
+
+
+def pin_embed_add_at(lib):
+    for seed, (N, L, K, H, skew) in enumerate([(200, 2, 9, 5, True), (64, 4, 31, 7, False)]):
+        ids, g = _embed_case(970 + seed, N, L, K, H, skew)
+        want = np.zeros((L, K, H))
+        for l in range(L):
+            np.add.at(want[l], ids[:, l], g.astype(np.float64))
+        got = oracle.embed_backward(ids, g, K, lib=lib)
+        assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def pin_embed_sums_and_bounds(lib):
+    ids, g = _embed_case(980, 400, 3, 20, 9, True)
+    grad, count, absum = oracle.embed_backward(ids, g, 20, bounds=True, lib=lib)
+    col = g.astype(np.float64).sum(axis=0)
+    for l in range(3):
+        assert np.allclose(grad[l].sum(axis=0), col, rtol=1e-12, atol=1e-12)
+        assert count[l].sum() == 400
+        assert np.array_equal(count[l], np.bincount(ids[:, l], minlength=20))
+    assert np.all(absum >= np.abs(grad) - 1e-12)
+    assert np.all(grad[count == 0] == 0.0)
+
+
 ALL_PINS = [pin_bruteforce, pin_nearest_neighbour_L1, pin_single_codeword,
             pin_codebook_equals_features, pin_ties_lowest_index, pin_invariants, pin_planted,
-            pin_decode_integer, pin_golden, pin_check_path]
+            pin_decode_integer, pin_golden, pin_check_path, pin_embed_adjoint, pin_embed_permutation,
+            pin_embed_add_at, pin_embed_sums_and_bounds]

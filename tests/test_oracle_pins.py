@@ -29,6 +29,11 @@ MUTANTS = {
     "skip_first_codeword": ("for (int k = 1; k < K; ++k) {\n        double d = sq_dist(r, C_l + (size_t)k * D, D);",
                             "bd = 1e300;\n    for (int k = 1; k < K; ++k) {\n        double d = sq_dist(r, C_l + (size_t)k * D, D);"),
     "square_dropped": ("s += t * t;", "s += t;"),
+    "embed_overwrites": ("for (int i = 0; i < H; ++i) dst[i] = dst[i] + (double)src[i];",
+                         "for (int i = 0; i < H; ++i) dst[i] = (double)src[i];"),
+    "embed_level0_ids": ("int32_t id = ids[(size_t)n * L + l];", "int32_t id = ids[(size_t)n * L];"),
+    "embed_transposed": ("double *dst = grad + ((size_t)l * K + (size_t)id) * H;",
+                         "double *dst = grad + ((size_t)id * L + (size_t)l) * H;"),
 }
 
 
