@@ -334,6 +334,34 @@ def run_ours(args, rank, world, local_rank):
     decode_bytes = N * L * 4 + rows_used * D * s_cb + N * D * 4
     decode_gbs = decode_bytes / (breakdown["decode"] / 1e3) / 1e9
 
+    # -------------------------------------------------- embedding backward (detok ids)
+    # The backbone's visual-token embedding e[n] = sum_l E_l[ids[n,l]] is the decode gather-sum
+    # with learned tables; its table gradient is the scatter-add grad[l, ids[n,l]] += g[n].  On
+    # the detok ids (level 0 Zipf-skewed) the decoded fp32 recon serves as a synthetic g [N,D],
+    # accumulated into fp32 tables [L,K,D] zeroed before each launch (outside the events).
+    embed = None
+    if detok_only:
+        gtab = torch.zeros((L, K, D), dtype=torch.float32, device=dev)
+        ev2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        eb = []
+        for _ in range(min(args.steps + 2, 6)):
+            gtab.zero_()
+            flush.zero_()
+            ev2[0].record(stream)
+            check(mvt.rvq_embed_backward(ids_in, N, L, K, D, rec2, gtab, status, stream), "rvq_embed_backward")
+            ev2[1].record(stream)
+            torch.cuda.synchronize(dev)
+            eb.append(ev2[0].elapsed_time(ev2[1]))
+        eb_ms = statistics.median(eb[1:]) if len(eb) > 1 else eb[0]
+        # algorithmic minimum: ids and g read once, every referenced gradient row read and written once
+        used = sum(int(np.unique(g["planted"][:, l]).size) for l in range(L))
+        eb_bytes = N * L * 4 + N * D * 4 + 2 * used * D * 4
+        embed = {"ms": eb_ms, "GB_per_s": eb_bytes / (eb_ms / 1e3) / 1e9, "algorithmic_bytes": eb_bytes,
+                 "frac_hbm": eb_bytes / (eb_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
+                 "fp32x4_atomics_per_s": N * L * (D // 4) / (eb_ms / 1e3),
+                 "g": "decoded fp32 recon [N,D]", "kernel": "embed_backward_kernel"}
+        del gtab
+
     # -------------------------------------------------- end to end through host buffers
     # Every step copies its features from pinned host memory and its ids + decoded recon back.
     # Two buffer sets and separate copy/compute streams let step k's copies overlap the compute of
@@ -456,6 +484,7 @@ def run_ours(args, rank, world, local_rank):
         "breakdown_ms": breakdown,
         "decode": {"GB_per_s": decode_gbs, "algorithmic_bytes": decode_bytes,
                    "frac_hbm": decode_gbs / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))},
+        **({"embed_backward": embed} if embed is not None else {}),
         "fallbacks_per_level": fb.cpu().tolist(),
         "parity_sample": parity,
     }

@@ -161,6 +161,24 @@ RVQ_API int rvq_decode(const int32_t *ids, int64_t N, int L, const void *codeboo
 RVQ_API const char *rvq_status_str(int status);
 
 /*
+ * rvq_embed_backward -- gradient of the backbone's visual-token embedding with respect to its
+ * tables (LongCat-2.5 technical blog, "Visual Primitive Modeling": the visual codebook embeddings
+ * are learned jointly with the backbone).  The embedding of token n is the decode gather-sum
+ * with learned tables E [L,K,H], e[n] = sum_l E_l[ids[n,l]] (rvq_decode with the tables computes
+ * it).  Given grad_out = dLoss/de [N,H] fp32 row-major, this adds, for every n and l,
+ *     grad_tables[l, ids[n,l], :] += grad_out[n, :]
+ * into grad_tables [L,K,H] fp32 row-major (the caller zeroes it for a fresh gradient; existing
+ * values are accumulated into).  Additions into one row arrive in no fixed order (fp32 atomics),
+ * so results can differ between runs by rounding, within (count - 1) * 2^-24 * sum of |terms|
+ * per element.  ids [N,L] int32.  An id outside [0, K) is skipped and RVQ_ERR_ID_RANGE goes to
+ * *status (optional device int32, first error wins).  All array pointers are caller-owned device
+ * pointers; grad_out and grad_tables 16-byte aligned.  Asynchronous on `stream`.
+ * Supported: N >= 0 (N = 0 is a no-op), 1 <= L <= 64, 1 <= K < 2^31, H % 4 == 0, H <= 65535 * 128.
+ */
+RVQ_API int rvq_embed_backward(const int32_t *ids, int64_t N, int L, int K, int H, const float *grad_out,
+                               float *grad_tables, int32_t *status, void *stream);
+
+/*
  * Measurement hooks (no counterpart on the pages).
  * rvq_launch_count: number of kernels this library has launched since it was loaded.
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on

@@ -27,7 +27,7 @@ STATUS = {0: "RVQ_OK", -1: "RVQ_ERR_ARG", -2: "RVQ_ERR_UNSUPPORTED", -3: "RVQ_ER
 
 EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
            "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read",
-           "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout",
+           "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
            "rvq_encode_noalloc")
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -69,9 +69,10 @@ def load(path: str | None = None):
         lib.rvq_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         lib.rvq_encode_levels_per_launch.argtypes = [i64, i32, i32, i32, ctypes.POINTER(i32)]
         lib.rvq_selftest_wait_timeout.argtypes = [vp, vp, i64, vp]
+        lib.rvq_embed_backward.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, vp]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
                    "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc",
-                   "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout"):
+                   "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -169,6 +170,11 @@ def rvq_encode_levels_per_launch(N, D, L, K):
     lv = ctypes.c_int32(0)
     code = load().rvq_encode_levels_per_launch(int(N), int(D), int(L), int(K), ctypes.byref(lv))
     return code, lv.value
+
+
+def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stream=None):
+    return load().rvq_embed_backward(_ptr(ids), int(N), int(L), int(K), int(H), _ptr(grad_out), _ptr(grad_tables),
+                                     _ptr(status), _stream(stream))
 
 
 def rvq_selftest_wait_timeout(counter, status, limit_us, stream=None):

@@ -75,6 +75,12 @@ def test_host_argument_checks(lib):
     assert L.rvq_encode_levels_per_launch(100, 1024, 4, 8192, None) == -1    # no output
     assert L.rvq_encode_levels_per_launch(100, 1000, 4, 8192, ctypes.byref(lv)) == -2   # D % 64
     assert L.rvq_encode_levels_per_launch(100, 1024, 65, 8192, ctypes.byref(lv)) == -2  # L > 64
+    eb = L.rvq_embed_backward
+    assert eb(16, 0, 2, 8, 64, 16, 16, None, None) == 0                        # N = 0: no-op
+    assert eb(None, 5, 2, 8, 64, 16, 16, None, None) == -1                     # no ids
+    assert eb(16, 5, 65, 8, 64, 16, 16, None, None) == -2                      # L > 64
+    assert eb(16, 5, 2, 8, 6, 16, 16, None, None) == -2                        # H % 4
+    assert eb(16, 5, 2, 8, 64, 24, 16, None, None) == -1                       # misaligned grad_out
     assert L.rvq_selftest_wait_timeout(None, 16, 1000, None) == -1               # no counter
     assert L.rvq_selftest_wait_timeout(16, 16, 0, None) == -1                  # limit out of range
 
