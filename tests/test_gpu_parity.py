@@ -117,6 +117,8 @@ EDGE = [
     (300, 1024, 1, 300, "f32", "f32"),      # all-levels kernel, one level
     (129, 1024, 3, 257, "bf16", "bf16"),    # all-levels kernel, two row tiles
     (2, 256, 4, 5000, "bf16", "f32"),       # all-levels kernel, one row tile
+    (300, 256, 20, 64, "f32", "f32"),       # all-levels kernel, 20 levels
+    (150, 1024, 64, 16, "bf16", "bf16"),    # all-levels kernel, the maximum 64 levels, K < 16
     (127, 64, 3, 300, "f32", "f32"),
     (129, 128, 2, 257, "bf16", "f32"),
     (300, 256, 2, 1, "f32", "f32"),
@@ -130,7 +132,8 @@ EDGE = [
 @pytest.mark.parametrize("N,D,L,K,fd,cd", EDGE)
 def test_edge_shapes(N, D, L, K, fd, cd):
     rng = np.random.Generator(np.random.PCG64([N, D, L, K]))
-    C = rng.standard_normal((L, K, D)).astype(np.float32) * (0.5 ** np.arange(L, dtype=np.float32))[:, None, None]
+    scale = 0.5 ** np.minimum(np.arange(L), 10).astype(np.float32)  # deep levels stay well inside fp32/bf16
+    C = rng.standard_normal((L, K, D)).astype(np.float32) * scale[:, None, None]
     x = rng.standard_normal((N, D)).astype(np.float32)
     if cd == "bf16":
         C = workloads.round_bf16(C)
