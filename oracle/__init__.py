@@ -64,6 +64,7 @@ def _declare(lib):
     lib.rvq_oracle_distances.argtypes = [f64p, f32p, I, I, f64p]
     lib.rvq_oracle_max_threads.argtypes = [I]
     lib.rvq_oracle_embed_backward.argtypes = [i32p, I64, I, I, I, f32p, f64p, i64p, f64p, I]
+    lib.rvq_oracle_codebook_update.argtypes = [f32p, i32p, I64, I, I, f32p, f64p, i64p, f64p]
     for fn in ("rvq_oracle_encode", "rvq_oracle_decode", "rvq_oracle_check_path",
                "rvq_oracle_distances", "rvq_oracle_max_threads"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -177,3 +178,25 @@ def embed_backward(ids, g, K, bounds: bool = False, threads: int = 0, lib=None):
     if rc != 0:
         raise OracleError(rc)
     return (grad, count, absum) if bounds else grad
+
+
+def codebook_update(points, ids, old_codebook, bounds: bool = False, lib=None):
+    """One k-means update of one level: new [K,D] fp64 (cluster means in ascending row order; an
+    empty cluster keeps its old codeword) and count [K]; with bounds=True also absum [K,D]."""
+    lib = lib or load()
+    points = _f32(points)
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    old = _f32(old_codebook)
+    N, D = points.shape
+    K, D2 = old.shape
+    assert D == D2 and ids.shape[0] == N
+    new = np.empty((K, D), np.float64)
+    count = np.empty(K, np.int64)
+    absum = np.empty((K, D), np.float64) if bounds else None
+    rc = lib.rvq_oracle_codebook_update(_p(points, ctypes.c_float), _p(ids, ctypes.c_int32), N, D, K,
+                                        _p(old, ctypes.c_float), _p(new, ctypes.c_double),
+                                        _p(count, ctypes.c_int64),
+                                        _p(absum, ctypes.c_double) if bounds else None)
+    if rc != 0:
+        raise OracleError(rc)
+    return (new, count, absum) if bounds else (new, count)

@@ -283,3 +283,50 @@ int rvq_oracle_embed_backward(const int32_t *ids, int64_t N, int L, int K, int H
     }
     return bad ? ORACLE_ERR_ID_RANGE : ORACLE_OK;
 }
+
+/*
+ * One Lloyd (k-means) update of one codebook level, the step that fits the fixed tokenizer the
+ * blog's "Offline Visual Preprocessing" relies on (the pages do not describe fitting; reading:
+ * plain k-means on the level's input residuals, an empty cluster keeps its codeword).  Given the
+ * level's input points p [N,D] (the residuals r_l the encode saw at this level) and their
+ * assignments ids [N] (the level's chosen codewords):
+ *     count[k]  = #{n : ids[n] == k}
+ *     new[k, :] = (1 / count[k]) * sum over those n of p[n, :]      (fp64, ascending n)
+ *     new[k, :] = old[k, :]                                           when count[k] == 0
+ * absum[k,:] (optional) = sum of |p[n,:]| over the cluster, for a rounding bound on an fp32 sum.
+ * An id outside [0, K) returns ORACLE_ERR_ID_RANGE and the row is ignored.
+ */
+int rvq_oracle_codebook_update(const float *p, const int32_t *ids, int64_t N, int D, int K, const float *old_cb,
+                               double *new_cb, int64_t *count, double *absum)
+{
+    if (!p || !ids || !old_cb || !new_cb || !count || D <= 0 || K <= 0 || N < 0) return ORACLE_ERR_ARG;
+    int bad = 0;
+    for (size_t i = 0; i < (size_t)K * D; ++i) new_cb[i] = 0.0;
+    if (absum)
+        for (size_t i = 0; i < (size_t)K * D; ++i) absum[i] = 0.0;
+    for (int k = 0; k < K; ++k) count[k] = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        int32_t id = ids[n];
+        if (id < 0 || id >= K) {
+            bad = 1;
+            continue;
+        }
+        double *s = new_cb + (size_t)id * D;
+        const float *x = p + (size_t)n * D;
+        for (int i = 0; i < D; ++i) s[i] = s[i] + (double)x[i];
+        if (absum) {
+            double *a = absum + (size_t)id * D;
+            for (int i = 0; i < D; ++i) a[i] = a[i] + fabs((double)x[i]);
+        }
+        count[id] += 1;
+    }
+    for (int k = 0; k < K; ++k) {
+        double *s = new_cb + (size_t)k * D;
+        if (count[k] == 0) {
+            for (int i = 0; i < D; ++i) s[i] = (double)old_cb[(size_t)k * D + i];
+        } else {
+            for (int i = 0; i < D; ++i) s[i] = s[i] / (double)count[k];
+        }
+    }
+    return bad ? ORACLE_ERR_ID_RANGE : ORACLE_OK;
+}

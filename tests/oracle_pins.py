@@ -16,7 +16,12 @@ learned tables) with:
   * the adjoint identity <decode(ids, E), G> = <E, backward(ids, G)> (decode pinned above),
   * a permutation of ids per level (each gradient row is one input row, exactly),
   * numpy's unbuffered scatter-add (np.add.at) on small inputs,
-  * column sums (every input row lands in exactly one row per level) and the magnitude bounds.
+  * column sums (every input row lands in exactly one row per level) and the magnitude bounds,
+and the k-means update of one codebook level with:
+  * points that are their own clusters (the codebook becomes the points, exactly),
+  * one cluster holding every point (numpy's mean),
+  * the Lloyd property: for fixed assignments the update never increases the squared error,
+  * numpy group-by means (bincount + add.at), empty clusters keeping their codeword.
 """
 from __future__ import annotations
 
@@ -291,7 +296,64 @@ def pin_embed_sums_and_bounds(lib):
     assert np.all(grad[count == 0] == 0.0)
 
 
+def pin_kmeans_own_clusters(lib):
+    rng = _rng(990)
+    N, D = 40, 6
+    p = rng.standard_normal((N, D)).astype(np.float32)
+    ids = rng.permutation(N).astype(np.int32)
+    old = rng.standard_normal((N, D)).astype(np.float32)
+    new, count = oracle.codebook_update(p, ids, old, lib=lib)
+    assert np.array_equal(count, np.ones(N, np.int64))
+    assert np.array_equal(new[ids], p.astype(np.float64))
+
+
+def pin_kmeans_single_cluster(lib):
+    rng = _rng(991)
+    p = rng.standard_normal((500, 9)).astype(np.float32)
+    old = rng.standard_normal((4, 9)).astype(np.float32)
+    new, count = oracle.codebook_update(p, np.full(500, 2, np.int32), old, lib=lib)
+    assert np.allclose(new[2], p.astype(np.float64).mean(axis=0), rtol=1e-13, atol=1e-15)
+    assert np.array_equal(new[[0, 1, 3]], old[[0, 1, 3]].astype(np.float64))
+    assert count.tolist() == [0, 0, 500, 0]
+
+
+def pin_kmeans_lloyd_step(lib):
+    rng = _rng(992)
+    N, D, K = 2000, 5, 30
+    p = rng.standard_normal((N, D)).astype(np.float32)
+    old = rng.standard_normal((K, D)).astype(np.float32)
+    ids, _, _, _ = oracle.encode(p, old[None], lib=lib)          # nearest codeword of each point
+    ids = ids[:, 0]
+    new, count = oracle.codebook_update(p, ids, old, lib=lib)
+    pd = p.astype(np.float64)
+    sse_old = float(((pd - old.astype(np.float64)[ids]) ** 2).sum())
+    sse_new = float(((pd - new[ids]) ** 2).sum())
+    assert sse_new <= sse_old * (1 + 1e-12), (sse_new, sse_old)
+    # and no other codeword set does better for these assignments: perturbing one mean hurts
+    k = int(np.argmax(count))
+    moved = new.copy()
+    moved[k] += 1e-3
+    assert float(((pd - moved[ids]) ** 2).sum()) > sse_new
+
+
+def pin_kmeans_groupby(lib):
+    rng = _rng(993)
+    N, D, K = 3000, 7, 64
+    p = rng.standard_normal((N, D)).astype(np.float32)
+    ids = np.minimum(rng.zipf(1.2, size=N) - 1, K - 9).astype(np.int32)   # skewed; the last 8 stay empty
+    old = rng.standard_normal((K, D)).astype(np.float32)
+    new, count = oracle.codebook_update(p, ids, old, lib=lib)
+    c = np.bincount(ids, minlength=K)
+    sums = np.zeros((K, D))
+    np.add.at(sums, ids, p.astype(np.float64))
+    want = np.where(c[:, None] > 0, sums / np.maximum(c, 1)[:, None], old.astype(np.float64))
+    assert np.array_equal(count, c)
+    assert (c == 0).any()
+    assert np.allclose(new, want, rtol=1e-13, atol=1e-15)
+
+
 ALL_PINS = [pin_bruteforce, pin_nearest_neighbour_L1, pin_single_codeword,
             pin_codebook_equals_features, pin_ties_lowest_index, pin_invariants, pin_planted,
             pin_decode_integer, pin_golden, pin_check_path, pin_embed_adjoint, pin_embed_permutation,
-            pin_embed_add_at, pin_embed_sums_and_bounds]
+            pin_embed_add_at, pin_embed_sums_and_bounds, pin_kmeans_own_clusters, pin_kmeans_single_cluster,
+            pin_kmeans_lloyd_step, pin_kmeans_groupby]

@@ -34,6 +34,12 @@ MUTANTS = {
     "embed_level0_ids": ("int32_t id = ids[(size_t)n * L + l];", "int32_t id = ids[(size_t)n * L];"),
     "embed_transposed": ("double *dst = grad + ((size_t)l * K + (size_t)id) * H;",
                          "double *dst = grad + ((size_t)id * L + (size_t)l) * H;"),
+    "kmeans_no_divide": ("for (int i = 0; i < D; ++i) s[i] = s[i] / (double)count[k];",
+                         "for (int i = 0; i < D; ++i) s[i] = s[i];"),
+    "kmeans_empty_zero": ("for (int i = 0; i < D; ++i) s[i] = (double)old_cb[(size_t)k * D + i];",
+                          "for (int i = 0; i < D; ++i) s[i] = 0.0;"),
+    "kmeans_skips_first_row": ("for (int64_t n = 0; n < N; ++n) {\n        int32_t id = ids[n];",
+                               "for (int64_t n = 1; n < N; ++n) {\n        int32_t id = ids[n];"),
 }
 
 
