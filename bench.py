@@ -334,6 +334,35 @@ def run_ours(args, rank, world, local_rank):
     decode_bytes = N * L * 4 + rows_used * D * s_cb + N * D * 4
     decode_gbs = decode_bytes / (breakdown["decode"] / 1e3) / 1e9
 
+    # -------------------------------------------------- k-means update of level 0 (offline)
+    # One Lloyd update of the level-0 codebook from the features and their level-0 ids: the step
+    # that fits the fixed tokenizer.  Points are the features widened to fp32 (outside the events).
+    kmeans = None
+    if args.workload == "offline":
+        pts = x.float()
+        ids0 = ids[:, 0].contiguous()
+        old0 = torch.from_numpy(np.ascontiguousarray(g["codebooks"][0], np.float32)).to(dev)
+        new0 = torch.empty_like(old0)
+        sums = torch.empty_like(old0)
+        cnt = torch.empty(K, dtype=torch.int32, device=dev)
+        ev3 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        km = []
+        for _ in range(min(args.steps + 2, 6)):
+            flush.zero_()
+            ev3[0].record(stream)
+            check(mvt.rvq_codebook_update(pts, ids0, N, D, K, old0, new0, sums, cnt, status, stream),
+                  "rvq_codebook_update")
+            ev3[1].record(stream)
+            torch.cuda.synchronize(dev)
+            km.append(ev3[0].elapsed_time(ev3[1]))
+        km_ms = statistics.median(km[1:])
+        # algorithmic minimum: points and ids read once, old codebook read, new codebook written
+        km_bytes = N * D * 4 + N * 4 + 2 * K * D * 4 + K * 4
+        kmeans = {"ms": km_ms, "GB_per_s": km_bytes / (km_ms / 1e3) / 1e9, "algorithmic_bytes": km_bytes,
+                  "frac_hbm": km_bytes / (km_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
+                  "level": 0, "kernels": "embed_backward_kernel (sums, counts) + kmeans_finalize_kernel"}
+        del pts, old0, new0, sums, cnt
+
     # -------------------------------------------------- embedding backward (detok ids)
     # The backbone's visual-token embedding e[n] = sum_l E_l[ids[n,l]] is the decode gather-sum
     # with learned tables; its table gradient is the scatter-add grad[l, ids[n,l]] += g[n].  On
@@ -485,6 +514,7 @@ def run_ours(args, rank, world, local_rank):
         "decode": {"GB_per_s": decode_gbs, "algorithmic_bytes": decode_bytes,
                    "frac_hbm": decode_gbs / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))},
         **({"embed_backward": embed} if embed is not None else {}),
+        **({"codebook_update": kmeans} if kmeans is not None else {}),
         "fallbacks_per_level": fb.cpu().tolist(),
         "parity_sample": parity,
     }

@@ -179,6 +179,26 @@ RVQ_API int rvq_embed_backward(const int32_t *ids, int64_t N, int L, int K, int 
                                float *grad_tables, int32_t *status, void *stream);
 
 /*
+ * rvq_codebook_update -- one k-means (Lloyd) update of one codebook level: the step that fits the
+ * fixed tokenizer whose ids the pages precompute offline (LongCat-2.5 technical blog, "Offline
+ * Visual Preprocessing"; the pages do not describe the fitting: plain k-means on the level's input
+ * residuals is the reading).  points [N,D] fp32 are the level's input residuals r_l (for level 0
+ * the features), ids [N] int32 their assigned codewords (the level's column of rvq_encode's ids,
+ * made contiguous).  For every k:
+ *     counts[k] = #{n : ids[n] == k}
+ *     new_codebook[k] = (sum of points[n] over those n) / counts[k]   (fp32 sum, any order)
+ *     new_codebook[k] = old_codebook[k]                                (counts[k] == 0)
+ * old_codebook, new_codebook [K,D] fp32 (they may be the same buffer: an in-place update); sums
+ * [K,D] fp32 is caller-owned scratch; counts [K] int32 is an output.  All are caller-owned device
+ * pointers, 16-byte aligned (counts, ids 4-byte).  Ids outside [0, K) are skipped and
+ * RVQ_ERR_ID_RANGE goes to *status (optional device int32).  Asynchronous on `stream`.
+ * Supported: 0 <= N < 2^31, D % 4 == 0, K >= 1.
+ */
+RVQ_API int rvq_codebook_update(const float *points, const int32_t *ids, int64_t N, int D, int K,
+                                const float *old_codebook, float *new_codebook, float *sums, int32_t *counts,
+                                int32_t *status, void *stream);
+
+/*
  * Measurement hooks (no counterpart on the pages).
  * rvq_launch_count: number of kernels this library has launched since it was loaded.
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on

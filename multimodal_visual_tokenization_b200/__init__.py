@@ -28,6 +28,7 @@ STATUS = {0: "RVQ_OK", -1: "RVQ_ERR_ARG", -2: "RVQ_ERR_UNSUPPORTED", -3: "RVQ_ER
 EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
            "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read",
            "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
+           "rvq_codebook_update",
            "rvq_encode_noalloc")
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -70,9 +71,11 @@ def load(path: str | None = None):
         lib.rvq_encode_levels_per_launch.argtypes = [i64, i32, i32, i32, ctypes.POINTER(i32)]
         lib.rvq_selftest_wait_timeout.argtypes = [vp, vp, i64, vp]
         lib.rvq_embed_backward.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, vp]
+        lib.rvq_codebook_update.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
                    "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc",
-                   "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward"):
+                   "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
+                   "rvq_codebook_update"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -175,6 +178,11 @@ def rvq_encode_levels_per_launch(N, D, L, K):
 def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stream=None):
     return load().rvq_embed_backward(_ptr(ids), int(N), int(L), int(K), int(H), _ptr(grad_out), _ptr(grad_tables),
                                      _ptr(status), _stream(stream))
+
+
+def rvq_codebook_update(points, ids, N, D, K, old_codebook, new_codebook, sums, counts, status=None, stream=None):
+    return load().rvq_codebook_update(_ptr(points), _ptr(ids), int(N), int(D), int(K), _ptr(old_codebook),
+                                      _ptr(new_codebook), _ptr(sums), _ptr(counts), _ptr(status), _stream(stream))
 
 
 def rvq_selftest_wait_timeout(counter, status, limit_us, stream=None):

@@ -81,6 +81,10 @@ def test_host_argument_checks(lib):
     assert eb(16, 5, 65, 8, 64, 16, 16, None, None) == -2                      # L > 64
     assert eb(16, 5, 2, 8, 6, 16, 16, None, None) == -2                        # H % 4
     assert eb(16, 5, 2, 8, 64, 24, 16, None, None) == -1                       # misaligned grad_out
+    cu = L.rvq_codebook_update
+    assert cu(16, 16, 5, 6, 8, 16, 16, 16, 16, None, None) == -2               # D % 4
+    assert cu(16, 16, 5, 64, 8, None, 16, 16, 16, None, None) == -1            # no old codebook
+    assert cu(24, 16, 5, 64, 8, 16, 16, 16, 16, None, None) == -1              # misaligned points
     assert L.rvq_selftest_wait_timeout(None, 16, 1000, None) == -1               # no counter
     assert L.rvq_selftest_wait_timeout(16, 16, 0, None) == -1                  # limit out of range
 
