@@ -65,6 +65,7 @@ def _declare(lib):
     lib.rvq_oracle_max_threads.argtypes = [I]
     lib.rvq_oracle_embed_backward.argtypes = [i32p, I64, I, I, I, f32p, f64p, i64p, f64p, I]
     lib.rvq_oracle_codebook_update.argtypes = [f32p, i32p, I64, I, I, f32p, f64p, i64p, f64p]
+    lib.rvq_oracle_balance.argtypes = [i64p, I64, I, i32p, i64p]
     for fn in ("rvq_oracle_encode", "rvq_oracle_decode", "rvq_oracle_check_path",
                "rvq_oracle_distances", "rvq_oracle_max_threads"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -200,3 +201,17 @@ def codebook_update(points, ids, old_codebook, bounds: bool = False, lib=None):
     if rc != 0:
         raise OracleError(rc)
     return (new, count, absum) if bounds else (new, count)
+
+
+def balance(lengths, world: int, lib=None):
+    """Longest-processing-time-first assignment of sequences to ranks: (owner [S], load [world])."""
+    lib = lib or load()
+    lengths = np.ascontiguousarray(lengths, dtype=np.int64)
+    S = lengths.shape[0]
+    owner = np.empty(S, np.int32)
+    ld = np.empty(world, np.int64)
+    rc = lib.rvq_oracle_balance(_p(lengths, ctypes.c_int64), S, int(world), _p(owner, ctypes.c_int32),
+                                _p(ld, ctypes.c_int64))
+    if rc != 0:
+        raise OracleError(rc)
+    return owner, ld

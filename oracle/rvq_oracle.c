@@ -330,3 +330,42 @@ int rvq_oracle_codebook_update(const float *p, const int32_t *ids, int64_t N, in
     }
     return bad ? ORACLE_ERR_ID_RANGE : ORACLE_OK;
 }
+
+/*
+ * Balance pretokenized image sequences across data-parallel ranks by visual-token count
+ * (LongCat-2.5 technical blog, "Offline Visual Preprocessing" and "Supernode-Aware Parallelism":
+ * with ids precomputed, every image's token count is known when batches are packed, which keeps
+ * the load even across data-parallel ranks; the pages give no algorithm, the reading is the
+ * classic longest-processing-time-first rule).  Sequences are taken in decreasing length (equal
+ * lengths: lower index first) and each goes to the rank with the smallest load so far (equal
+ * loads: lower rank).  owner[s] receives the rank of sequence s, load[r] the tokens of rank r.
+ * Plain O(S log S + S * world) loops.
+ */
+int rvq_oracle_balance(const int64_t *lengths, int64_t S, int world, int32_t *owner, int64_t *load)
+{
+    if (!lengths || !owner || !load || S < 0 || world < 1) return ORACLE_ERR_ARG;
+    for (int64_t s = 0; s < S; ++s)
+        if (lengths[s] < 0) return ORACLE_ERR_ARG;
+    int64_t *order = (int64_t *)malloc((size_t)(S > 0 ? S : 1) * sizeof(int64_t));
+    if (!order) return ORACLE_ERR_ARG;
+    for (int64_t s = 0; s < S; ++s) order[s] = s;
+    /* insertion sort: decreasing length, then increasing index (stable on the index order) */
+    for (int64_t i = 1; i < S; ++i) {
+        int64_t v = order[i], j = i - 1;
+        while (j >= 0 && lengths[order[j]] < lengths[v]) {
+            order[j + 1] = order[j];
+            --j;
+        }
+        order[j + 1] = v;
+    }
+    for (int r = 0; r < world; ++r) load[r] = 0;
+    for (int64_t i = 0; i < S; ++i) {
+        int best = 0;
+        for (int r = 1; r < world; ++r)
+            if (load[r] < load[best]) best = r;
+        owner[order[i]] = best;
+        load[best] += lengths[order[i]];
+    }
+    free(order);
+    return ORACLE_OK;
+}

@@ -21,7 +21,12 @@ and the k-means update of one codebook level with:
   * points that are their own clusters (the codebook becomes the points, exactly),
   * one cluster holding every point (numpy's mean),
   * the Lloyd property: for fixed assignments the update never increases the squared error,
-  * numpy group-by means (bincount + add.at), empty clusters keeping their codeword.
+  * numpy group-by means (bincount + add.at), empty clusters keeping their codeword,
+and the balance of sequences across data-parallel ranks with:
+  * brute force over all assignments on tiny inputs (Graham's bound for the longest-first rule:
+    max load <= (4/3 - 1/(3 world)) x the optimum, and never below it),
+  * the hand-worked example in tests/golden/lpt_balance.txt,
+  * invariants (every sequence owned once, loads add up, equal lengths split evenly).
 """
 from __future__ import annotations
 
@@ -352,8 +357,41 @@ def pin_kmeans_groupby(lib):
     assert np.allclose(new, want, rtol=1e-13, atol=1e-15)
 
 
+def pin_balance_bruteforce(lib):
+    rng = _rng(994)
+    for _ in range(40):
+        S = int(rng.integers(1, 8))
+        world = int(rng.integers(1, 4))
+        lengths = rng.integers(0, 50, size=S)
+        owner, load = oracle.balance(lengths, world, lib=lib)
+        assert owner.min() >= 0 and owner.max() < world
+        assert np.array_equal(load, np.bincount(owner, weights=lengths, minlength=world).astype(np.int64))
+        best = min(max(np.bincount(np.array(a), weights=lengths, minlength=world))
+                   for a in itertools.product(range(world), repeat=S))
+        assert best <= load.max() <= (4.0 / 3.0 - 1.0 / (3 * world)) * best + 1e-9, (lengths, world, load, best)
+
+
+def pin_balance_golden(lib):
+    vals = {}
+    with open(os.path.join(GOLDEN, "lpt_balance.txt")) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                k, *v = ln.split()
+                vals[k] = [int(t) for t in v]
+    owner, load = oracle.balance(vals["lengths"], vals["world"][0], lib=lib)
+    assert owner.tolist() == vals["owner"] and load.tolist() == vals["load"]
+
+
+def pin_balance_invariants(lib):
+    owner, load = oracle.balance(np.full(100, 37), 8, lib=lib)
+    assert load.max() - load.min() <= 37 and load.sum() == 3700
+    owner, load = oracle.balance(np.arange(500), 1, lib=lib)
+    assert (owner == 0).all() and load.tolist() == [sum(range(500))]
+
+
 ALL_PINS = [pin_bruteforce, pin_nearest_neighbour_L1, pin_single_codeword,
             pin_codebook_equals_features, pin_ties_lowest_index, pin_invariants, pin_planted,
             pin_decode_integer, pin_golden, pin_check_path, pin_embed_adjoint, pin_embed_permutation,
             pin_embed_add_at, pin_embed_sums_and_bounds, pin_kmeans_own_clusters, pin_kmeans_single_cluster,
-            pin_kmeans_lloyd_step, pin_kmeans_groupby]
+            pin_kmeans_lloyd_step, pin_kmeans_groupby, pin_balance_bruteforce, pin_balance_golden,
+            pin_balance_invariants]

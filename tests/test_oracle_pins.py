@@ -40,6 +40,9 @@ MUTANTS = {
                           "for (int i = 0; i < D; ++i) s[i] = 0.0;"),
     "kmeans_skips_first_row": ("for (int64_t n = 0; n < N; ++n) {\n        int32_t id = ids[n];",
                                "for (int64_t n = 1; n < N; ++n) {\n        int32_t id = ids[n];"),
+    "balance_most_loaded": ("if (load[r] < load[best]) best = r;", "if (load[r] > load[best]) best = r;"),
+    "balance_increasing": ("while (j >= 0 && lengths[order[j]] < lengths[v]) {",
+                           "while (j >= 0 && lengths[order[j]] > lengths[v]) {"),
 }
 
 
