@@ -370,6 +370,37 @@ def run_ours(args, rank, world, local_rank):
                   "level": 0, "kernels": "embed_backward_kernel (sums, counts) + kmeans_finalize_kernel"}
         del pts, old0, new0, sums, cnt
 
+    # -------------------------------------------------- packing for data-parallel ranks (packed)
+    # The batch's images balanced over 8 ranks by token count (host), then every rank's share
+    # gathered from the id cache (the ids just computed) into rank-major packed order (GPU).
+    pack = None
+    if args.workload == "packed":
+        lengths = np.diff(g["offsets"])
+        code, owner, pload = mvt.rvq_balance_sequences(lengths, 8)
+        check(code, "rvq_balance_sequences")
+        select = np.concatenate([np.nonzero(owner == r)[0] for r in range(8)]).astype(np.int64)
+        out_off = np.concatenate([[0], np.cumsum(lengths[select])]).astype(np.int64)
+        sel_d = torch.from_numpy(select).to(dev)
+        oo_d = torch.from_numpy(out_off).to(dev)
+        packed_ids = torch.empty_like(ids)
+        ev4 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        pk = []
+        for _ in range(6):
+            flush_l2()
+            ev4[0].record(stream)
+            check(mvt.rvq_gather_sequences(ids, L, off, B, sel_d, B, oo_d, packed_ids, status, stream),
+                  "rvq_gather_sequences")
+            ev4[1].record(stream)
+            torch.cuda.synchronize(dev)
+            pk.append(ev4[0].elapsed_time(ev4[1]))
+        pk_ms = statistics.median(pk[1:])
+        pk_bytes = 2 * N * L * 4 + B * 8 * 3
+        pack = {"ms": pk_ms, "GB_per_s": pk_bytes / (pk_ms / 1e3) / 1e9, "algorithmic_bytes": pk_bytes,
+                "frac_hbm": pk_bytes / (pk_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
+                "world": 8, "images": int(B), "max_over_mean_rank_tokens": float(pload.max() / pload.mean()),
+                "kernel": "gather_sequences_kernel"}
+        del packed_ids
+
     # -------------------------------------------------- embedding backward (detok ids)
     # The backbone's visual-token embedding e[n] = sum_l E_l[ids[n,l]] is the decode gather-sum
     # with learned tables; its table gradient is the scatter-add grad[l, ids[n,l]] += g[n].  On
@@ -521,6 +552,7 @@ def run_ours(args, rank, world, local_rank):
         "decode": {"GB_per_s": decode_gbs, "algorithmic_bytes": decode_bytes,
                    "frac_hbm": decode_gbs / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))},
         **({"embed_backward": embed} if embed is not None else {}),
+        **({"pack": pack} if pack is not None else {}),
         **({"codebook_update": kmeans} if kmeans is not None else {}),
         "fallbacks_per_level": fb.cpu().tolist(),
         "parity_sample": parity,

@@ -199,6 +199,33 @@ RVQ_API int rvq_codebook_update(const float *points, const int32_t *ids, int64_t
                                 int32_t *status, void *stream);
 
 /*
+ * Packing pretokenized image sequences for data-parallel ranks (LongCat-2.5 technical blog,
+ * "Offline Visual Preprocessing" and "Supernode-Aware Parallelism": with the ids precomputed,
+ * every image's token count is known when batches are packed, which keeps the load even across
+ * data-parallel ranks; the pages give no algorithm).
+ *
+ * rvq_balance_sequences (host only, no GPU): assigns S sequences of lengths[S] (>= 0 tokens) to
+ * `world` ranks, longest processing time first: sequences in decreasing length (equal lengths:
+ * lower index first) each go to the least-loaded rank so far (equal loads: lower rank), so every
+ * rank computes the same assignment from the same lengths.  owner[S] receives the rank of each
+ * sequence, load[world] each rank's total tokens; the largest load is at most
+ * (4/3 - 1/(3 world)) times the best possible.  Host pointers.  RVQ_ERR_ARG on bad arguments.
+ *
+ * rvq_gather_sequences (GPU): packs the id rows of M selected sequences out of an id cache.
+ * cache_ids [T, L] int32 holds the ids of all cached sequences back to back, sequence s being rows
+ * [cache_offsets[s], cache_offsets[s+1]) (cache_offsets [S+1], int64); select [M] int64 lists the
+ * sequences to pack; out_offsets [M+1] int64 gives where each lands in out_ids [out_offsets[M], L]
+ * (prefix sums of the selected lengths, computed by the caller, who knows them from the balance).
+ * A selected index outside [0, S) or an out_offsets span that differs from the cached length is
+ * skipped and RVQ_ERR_ARG goes to *status (optional device int32).  All array pointers are
+ * caller-owned device pointers.  Asynchronous on `stream`.  Supported: M < 2^31.
+ */
+RVQ_API int rvq_balance_sequences(const int64_t *lengths, int64_t S, int world, int32_t *owner, int64_t *load);
+RVQ_API int rvq_gather_sequences(const int32_t *cache_ids, int L, const int64_t *cache_offsets, int64_t S,
+                                 const int64_t *select, int64_t M, const int64_t *out_offsets, int32_t *out_ids,
+                                 int32_t *status, void *stream);
+
+/*
  * Measurement hooks (no counterpart on the pages).
  * rvq_launch_count: number of kernels this library has launched since it was loaded.
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on

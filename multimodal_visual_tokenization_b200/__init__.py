@@ -28,7 +28,7 @@ STATUS = {0: "RVQ_OK", -1: "RVQ_ERR_ARG", -2: "RVQ_ERR_UNSUPPORTED", -3: "RVQ_ER
 EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
            "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read",
            "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
-           "rvq_codebook_update",
+           "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
            "rvq_encode_noalloc")
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -72,10 +72,12 @@ def load(path: str | None = None):
         lib.rvq_selftest_wait_timeout.argtypes = [vp, vp, i64, vp]
         lib.rvq_embed_backward.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, vp]
         lib.rvq_codebook_update.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+        lib.rvq_balance_sequences.argtypes = [vp, i64, i32, vp, vp]
+        lib.rvq_gather_sequences.argtypes = [vp, i32, vp, i64, vp, i64, vp, vp, vp, vp]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
                    "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc",
                    "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
-                   "rvq_codebook_update"):
+                   "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -183,6 +185,22 @@ def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stre
 def rvq_codebook_update(points, ids, N, D, K, old_codebook, new_codebook, sums, counts, status=None, stream=None):
     return load().rvq_codebook_update(_ptr(points), _ptr(ids), int(N), int(D), int(K), _ptr(old_codebook),
                                       _ptr(new_codebook), _ptr(sums), _ptr(counts), _ptr(status), _stream(stream))
+
+
+def rvq_balance_sequences(lengths, world):
+    """Host call: lengths is a sequence of token counts; returns (code, owner [S] int32, load [world] int64)."""
+    import numpy as np
+    lengths = np.ascontiguousarray(lengths, dtype=np.int64)
+    owner = np.empty(lengths.shape[0], np.int32)
+    load_ = np.empty(int(world), np.int64)
+    code = load().rvq_balance_sequences(lengths.ctypes.data if lengths.size else None, lengths.shape[0], int(world),
+                                        owner.ctypes.data, load_.ctypes.data)
+    return code, owner, load_
+
+
+def rvq_gather_sequences(cache_ids, L, cache_offsets, S, select, M, out_offsets, out_ids, status=None, stream=None):
+    return load().rvq_gather_sequences(_ptr(cache_ids), int(L), _ptr(cache_offsets), int(S), _ptr(select), int(M),
+                                       _ptr(out_offsets), _ptr(out_ids), _ptr(status), _stream(stream))
 
 
 def rvq_selftest_wait_timeout(counter, status, limit_us, stream=None):

@@ -85,6 +85,9 @@ def test_host_argument_checks(lib):
     assert cu(16, 16, 5, 6, 8, 16, 16, 16, 16, None, None) == -2               # D % 4
     assert cu(16, 16, 5, 64, 8, None, 16, 16, 16, None, None) == -1            # no old codebook
     assert cu(24, 16, 5, 64, 8, 16, 16, 16, 16, None, None) == -1              # misaligned points
+    assert L.rvq_gather_sequences(16, 0, 16, 1, 16, 1, 16, 16, None, None) == -1   # L < 1
+    assert L.rvq_gather_sequences(16, 8, 16, 1, 16, 0, 16, 16, None, None) == 0    # M = 0: no-op
+    assert L.rvq_gather_sequences(None, 8, 16, 1, 16, 1, 16, 16, None, None) == -1 # no cache
     assert L.rvq_selftest_wait_timeout(None, 16, 1000, None) == -1               # no counter
     assert L.rvq_selftest_wait_timeout(16, 16, 0, None) == -1                  # limit out of range
 
