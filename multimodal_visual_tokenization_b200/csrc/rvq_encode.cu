@@ -1307,6 +1307,11 @@ constexpr int FLOW_EPI_WIDE = 8;
 constexpr int FLOW_RW_WIDE = 5;
 constexpr int FLOW_EPI_NARROW = 8;
 constexpr int FLOW_RW_NARROW = 5;
+// Idle warps among the five (bit i = warp CERT0 + i): at D = 1024 warp 13, which shares the MMA
+// issuer's sub-partition (4 certificate warps; image 13.2 vs 13.1 Mtok/s with 5, 12.8 with 3);
+// at D = 256 also warp 12, the TMA producer's (3 certificate warps; offline 7.61 vs 7.45 with 4).
+constexpr int FLOW_SKIP_WIDE = 0b00100;
+constexpr int FLOW_SKIP_NARROW = 0b00110;
 constexpr int EXACT_QCAP = 1024;   // queued rows whose exact scan is split into slices
 constexpr int EXACT_NS_MAX = 256;  // codeword slices per queued row
 
@@ -1440,20 +1445,25 @@ __device__ __forceinline__ void exact_slice(const RowArgs &a, int64_t n, int k0,
   }
 }
 
-template <int EPI, int RW>
+// RW warps follow the GEMM roles; those in the bit mask SKIP (relative to CERT0) stay idle, so that
+// no certificate work shares a scheduler sub-partition (warp w runs on sub-partition w % 4) with
+// the MMA issuer or, when set, the TMA producer.
+template <int EPI, int RW, int SKIP>
 struct FlowCfg {
   static constexpr int THREADS = GemmCfg<EPI, false>::THREADS + RW * 32;
-  static constexpr int CERT0 = EPI + 3;  // first certificate warp
+  static constexpr int CERT0 = EPI + 3;  // first of the RW warps after the GEMM roles
+  static constexpr int CERT_WARPS = RW - __builtin_popcount(SKIP);
 };
 
-template <int EPI, int RW, bool CB_BF16, bool X_BF16, int NCH>
-__global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
+template <int EPI, int RW, int SKIP, bool CB_BF16, bool X_BF16, int NCH>
+__global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     encode_flow_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB3, const GemmArgs a, const RowArgs r0,
                        const FlowArgs fa) {
   using C = GemmCfg<EPI, false>;
   constexpr int NSTAGE = C::NSTAGE;
-  constexpr int CERT0 = FlowCfg<EPI, RW>::CERT0;
+  constexpr int CERT0 = FlowCfg<EPI, RW, SKIP>::CERT0;
+  constexpr int CW = FlowCfg<EPI, RW, SKIP>::CERT_WARPS;
   constexpr int SRC0 = X_BF16 ? SRC_X_BF16 : SRC_X_F32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1799,10 +1809,11 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW>::THREADS, 1)
       *abort_flag = 1;
       set_status(a.status, RVQ_ERR_TIMEOUT);
     }
-  } else if (warp >= CERT0) {
+  } else if (warp >= CERT0 && !((SKIP >> (warp - CERT0)) & 1)) {
     // ------------------------------------------------------------ certificate warps
-    const int64_t cw = static_cast<int64_t>(G) * RW;
-    const int64_t gw = static_cast<int64_t>(blockIdx.x) * RW + (warp - CERT0);
+    const int64_t cw = static_cast<int64_t>(G) * CW;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * CW + (warp - CERT0) -
+                       __popc(SKIP & ((1u << (warp - CERT0)) - 1u));
     const int TG = BM / fa.RPT;
     const int64_t total_tasks = static_cast<int64_t>(fa.L) * RT * TG;
     const uint32_t all_rows = static_cast<uint32_t>(a.N) * static_cast<uint32_t>(fa.L);
@@ -2119,7 +2130,8 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
     p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
     p.maxs = std::max(p.maxs, p.NC);
     // certificate tasks: about two per certificate warp per level, at most one row tile each
-    const int64_t cw = static_cast<int64_t>(p.Gf) * (nch == 8 ? FLOW_RW_WIDE : FLOW_RW_NARROW);
+    const int64_t cw = static_cast<int64_t>(p.Gf) * (nch == 8 ? FlowCfg<FLOW_EPI_WIDE, FLOW_RW_WIDE, FLOW_SKIP_WIDE>::CERT_WARPS
+                                                              : FlowCfg<FLOW_EPI_NARROW, FLOW_RW_NARROW, FLOW_SKIP_NARROW>::CERT_WARPS);
     int tg = 1;
     while (tg < 64 && static_cast<int64_t>(tg) * p.RT < 2 * cw) tg *= 2;
     p.RPT = BM / tg;
@@ -2289,31 +2301,32 @@ inline int resident_pair_clusters(int D) {
 // All-levels dataflow encode, instantiated for 2 (D in (128, 256]) and 8 (D in (512, 1024])
 // float4 row chunks.
 
-template <int EPI, int RW, bool CB, bool XB, int NCH>
+template <int EPI, int RW, int SK, bool CB, bool XB, int NCH>
 inline bool set_flow_attr() {
-  return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, CB, XB, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<EPI, false>::SMEM) == cudaSuccess;
+  return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, SK, CB, XB, NCH>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<EPI, false>::SMEM) == cudaSuccess;
 }
 
 inline bool flow_attrs_ready() {
   static std::once_flag once;
   static bool ok = false;
   std::call_once(once, [] {
-    constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW;
-    ok = set_flow_attr<EW, RWD, false, false, 8>() && set_flow_attr<EW, RWD, false, true, 8>() &&
-         set_flow_attr<EW, RWD, true, false, 8>() && set_flow_attr<EW, RWD, true, true, 8>() &&
-         set_flow_attr<EN, RN, false, false, 2>() && set_flow_attr<EN, RN, false, true, 2>() &&
-         set_flow_attr<EN, RN, true, false, 2>() && set_flow_attr<EN, RN, true, true, 2>();
+    constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, SW = FLOW_SKIP_WIDE;
+    constexpr int EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW, SN = FLOW_SKIP_NARROW;
+    ok = set_flow_attr<EW, RWD, SW, false, false, 8>() && set_flow_attr<EW, RWD, SW, false, true, 8>() &&
+         set_flow_attr<EW, RWD, SW, true, false, 8>() && set_flow_attr<EW, RWD, SW, true, true, 8>() &&
+         set_flow_attr<EN, RN, SN, false, false, 2>() && set_flow_attr<EN, RN, SN, false, true, 2>() &&
+         set_flow_attr<EN, RN, SN, true, false, 2>() && set_flow_attr<EN, RN, SN, true, true, 2>();
   });
   return ok;
 }
 
-template <int EPI, int RW, bool CB, bool XB, int NCH>
+template <int EPI, int RW, int SK, bool CB, bool XB, int NCH>
 inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tmA0, const CUtensorMap &tmA,
                                  const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(FlowCfg<EPI, RW>::THREADS);
+  cfg.blockDim = dim3(FlowCfg<EPI, RW, SK>::THREADS);
   cfg.dynamicSmemBytes = GemmCfg<EPI, false>::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -2321,24 +2334,25 @@ inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tm
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, CB, XB, NCH>, tmA0, tmA, tmB3, ga, ra, fa);
+  return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, SK, CB, XB, NCH>, tmA0, tmA, tmB3, ga, ra, fa);
 }
 
 inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cudaStream_t s, const CUtensorMap &tmA0,
                                const CUtensorMap &tmA, const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra,
                                const FlowArgs &fa) {
-  constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW;
+  constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, SW = FLOW_SKIP_WIDE;
+  constexpr int EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW, SN = FLOW_SKIP_NARROW;
   if (nch == 2) {
-    if (cb_bf16) return x_bf16 ? launch_flow_t<EN, RN, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                               : launch_flow_t<EN, RN, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
-    return x_bf16 ? launch_flow_t<EN, RN, false, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                  : launch_flow_t<EN, RN, false, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    if (cb_bf16) return x_bf16 ? launch_flow_t<EN, RN, SN, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                               : launch_flow_t<EN, RN, SN, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    return x_bf16 ? launch_flow_t<EN, RN, SN, false, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                  : launch_flow_t<EN, RN, SN, false, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
   }
   if (nch != 8) return cudaErrorInvalidValue;
-  if (cb_bf16) return x_bf16 ? launch_flow_t<EW, RWD, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                             : launch_flow_t<EW, RWD, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
-  return x_bf16 ? launch_flow_t<EW, RWD, false, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
-                : launch_flow_t<EW, RWD, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  if (cb_bf16) return x_bf16 ? launch_flow_t<EW, RWD, SW, true, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                             : launch_flow_t<EW, RWD, SW, true, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  return x_bf16 ? launch_flow_t<EW, RWD, SW, false, true, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                : launch_flow_t<EW, RWD, SW, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
 }
 
 inline cudaError_t launch_gemm(int epi, bool pair, int groups, cudaStream_t s, const CUtensorMap &tmA,
