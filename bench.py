@@ -370,6 +370,41 @@ def run_ours(args, rank, world, local_rank):
                   "level": 0, "kernels": "embed_backward_kernel (sums, counts) + kmeans_finalize_kernel"}
         del pts, old0, new0, sums, cnt
 
+    # -------------------------------------------------- codebook-sharded encode (image)
+    # The codebook axis split in two shards that this one GPU both holds (one process standing in
+    # for two ranks, so the exchange of (distance, id) pairs is empty): per level a distance GEMM
+    # over each half, the shards' certificates and the apply kernel.  The ids must equal the
+    # one-GPU encode's; the GEMM launches are timed with the profiling events.
+    sharded = None
+    if args.workload == "image" and world == 1:
+        from multimodal_visual_tokenization_b200.sharded import ShardedTokenizer
+        stok = ShardedTokenizer.local(cb, 2)
+        for _ in range(2):
+            stok.encode(x, status=status)
+        ev5 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        sh = []
+        mvt.rvq_profile_enable(True)
+        for _ in range(6):
+            flush_l2()
+            ev5[0].record(stream)
+            sids, _, sfb = stok.encode(x, status=status)
+            ev5[1].record(stream)
+            torch.cuda.synchronize(dev)
+            sh.append(ev5[0].elapsed_time(ev5[1]))
+        code, sg_n, sg_ms = mvt.rvq_profile_read()
+        mvt.rvq_profile_enable(False)
+        sh_ms = statistics.median(sh)
+        sg_tflops = 6 * 2.0 * N * K * D * L / (sg_ms / 1e3) / 1e12 if sg_ms > 0 else None
+        sharded = {"shards": 2, "ms": sh_ms, "Mtok_per_s": N / (sh_ms / 1e3) / 1e6,
+                   "ids_equal_one_gpu": bool(torch.equal(sids, ids)),
+                   "gemm_tflops": sg_tflops,
+                   "gemm_frac": (sg_tflops / float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+                                 if sg_tflops else None),
+                   "fallback_rows": int(sfb.sum().item()),
+                   "kernels": "dist_topk_kernel per shard + shard_select/fallback + shard_apply",
+                   "note": "both shards on one GPU; exchange empty"}
+        del stok
+
     # -------------------------------------------------- packing for data-parallel ranks (packed)
     # The batch's images balanced over 8 ranks by token count (host), then every rank's share
     # gathered from the id cache (the ids just computed) into rank-major packed order (GPU).
@@ -553,6 +588,7 @@ def run_ours(args, rank, world, local_rank):
                    "frac_hbm": decode_gbs / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))},
         **({"embed_backward": embed} if embed is not None else {}),
         **({"pack": pack} if pack is not None else {}),
+        **({"sharded": sharded} if sharded is not None else {}),
         **({"codebook_update": kmeans} if kmeans is not None else {}),
         "fallbacks_per_level": fb.cpu().tolist(),
         "parity_sample": parity,

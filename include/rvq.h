@@ -226,6 +226,67 @@ RVQ_API int rvq_gather_sequences(const int32_t *cache_ids, int L, const int64_t 
                                  int32_t *status, void *stream);
 
 /*
+ * Codebook-sharded encode: the same greedy RVQ as rvq_encode, with the codebook axis split over W
+ * ranks (one process per GPU) for codebook sets larger than one GPU holds.  The pages only fix the
+ * quantizer (LongCat-2.5 technical blog, "Discrete Native Resolution Vision Transformer": residual
+ * levels of nearest codewords); the split is this library's.  Rank w holds codewords
+ * [k0_w, k0_w + K_w) of every level, k0_w = K_0 + ... + K_{w-1}, as its own [L, K_w, D] array with
+ * norms / level statistics / operand copy from rvq_build_norms on that array, and every rank holds
+ * all N feature rows.  Per level l, in this order on every rank:
+ *   1. rvq_shard_select: this shard's nearest codeword for every row, with its exact distance,
+ *      into sel [N, 2] fp64 = (||r - c||^2 as an fp64 sum of fp32 differences, global id).  Same
+ *      candidate / certificate / exact-rescan scheme as rvq_encode, restricted to the shard.
+ *   2. the caller gathers every rank's sel into sel_all [W, N, 2] (rank w's at row block w), e.g.
+ *      an all-gather over the ranks' process group.
+ *   3. rvq_shard_apply: per row the lowest (distance, id) of sel_all is the level's id; ids[n, l]
+ *      receives it and the residual is updated with that codeword, read from its owner's array.
+ * The residual state lives in the workspace (or in `residual`, when given), so one rank's calls of
+ * one encode share workspace and residual pointer, and every rank's state stays bit-identical.  The
+ * ids equal rvq_encode's for the whole codebook set (exact distances; ties to the lowest id).
+ *
+ * rvq_shard_workspace_size: device bytes for this rank (N rows, width D, K_shard codewords).
+ * rvq_shard_select: features [N, D] (f_dtype; read at l = 0), this rank's shard_codebooks
+ *   [L, K_shard, D] in cb_dtype, shard_operand (bf16 copy, NULL for RVQ_BF16), shard_norms [L,
+ *   K_shard] and shard_stats [L, RVQ_LEVEL_STATS] from rvq_build_norms of the shard; k0 = the
+ *   shard's first global id; residual optional [N, D] fp32 (the residual after the level applied
+ *   last); sel [N, 2] fp64 out; fallbacks optional [L] int32 device, entry l = rows of this level
+ *   that needed an exact scan of the shard.  Device pointers 16-byte aligned; workspace 256-byte.
+ * rvq_shard_apply: sel_all [W, N, 2] fp64; shard_codebooks = HOST array of W device pointers, entry
+ *   w pointing at rank w's [L, K_w, D] stored codebooks (a pointer from rvq_ipc_import for another
+ *   GPU's array); shard_K host array [W]; ids [N, L] int32 out (column l); residual as for select.
+ *   A row whose sel entries are all unusable (non-finite inputs) gets id -1 and RVQ_ERR_ARG in
+ *   *status.
+ * Both: asynchronous on `stream`; argument errors are returned before anything is enqueued.
+ * Supported: 64 <= D <= 1024, D % 64 == 0, 1 <= L <= 64, N < 2^31, 1 <= W <= RVQ_MAX_SHARDS,
+ * total K < 2^31.
+ */
+#define RVQ_MAX_SHARDS 16
+RVQ_API int rvq_shard_workspace_size(int64_t N, int D, int K_shard, size_t *bytes);
+RVQ_API int rvq_shard_select(const void *features, int f_dtype, int64_t N, int D, const void *shard_codebooks,
+                             int cb_dtype, const void *shard_operand, const float *shard_norms,
+                             const float *shard_stats, int L, int K_shard, int64_t k0, int l, float *residual,
+                             double *sel, int32_t *fallbacks, void *workspace, size_t workspace_bytes,
+                             int32_t *status, void *stream);
+RVQ_API int rvq_shard_apply(const void *features, int f_dtype, int64_t N, int D, const double *sel_all, int W,
+                            const void *const *shard_codebooks, int cb_dtype, const int *shard_K, int L, int l,
+                            int32_t *ids, float *residual, void *workspace, size_t workspace_bytes,
+                            int32_t *status, void *stream);
+
+/*
+ * Device buffers shared between the processes of one node (CUDA IPC), for rvq_shard_apply's
+ * peer pointers.  rvq_ipc_export: the RVQ_IPC_HANDLE_BYTES-byte handle of the device allocation
+ * that holds ptr, and ptr's byte offset in it (host outputs).  rvq_ipc_import (another process):
+ * maps that allocation on the current device (peer access enabled on first use) and returns
+ * *ptr = its base + offset; the mapping stays valid while the exporting process keeps the
+ * allocation.  rvq_ipc_close(ptr, offset) unmaps it.  RVQ_ERR_ARG for a pointer that is not
+ * device memory, RVQ_ERR_CUDA when the runtime refuses (e.g. import in the exporting process).
+ */
+#define RVQ_IPC_HANDLE_BYTES 64
+RVQ_API int rvq_ipc_export(const void *ptr, void *handle, size_t *offset);
+RVQ_API int rvq_ipc_import(const void *handle, size_t offset, void **ptr);
+RVQ_API int rvq_ipc_close(void *ptr, size_t offset);
+
+/*
  * Measurement hooks (no counterpart on the pages).
  * rvq_launch_count: number of kernels this library has launched since it was loaded.
  * rvq_profile_enable(1): from now on, bracket every distance-GEMM launch with CUDA events on

@@ -29,7 +29,10 @@ EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_de
            "rvq_status_str", "rvq_launch_count", "rvq_profile_enable", "rvq_profile_read",
            "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
            "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
-           "rvq_encode_noalloc")
+           "rvq_encode_noalloc", "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply",
+           "rvq_ipc_export", "rvq_ipc_import", "rvq_ipc_close")
+RVQ_MAX_SHARDS = 16
+RVQ_IPC_HANDLE_BYTES = 64
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _lib = None
@@ -74,10 +77,20 @@ def load(path: str | None = None):
         lib.rvq_codebook_update.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
         lib.rvq_balance_sequences.argtypes = [vp, i64, i32, vp, vp]
         lib.rvq_gather_sequences.argtypes = [vp, i32, vp, i64, vp, i64, vp, vp, vp, vp]
+        lib.rvq_shard_workspace_size.argtypes = [i64, i32, i32, ctypes.POINTER(sz)]
+        lib.rvq_shard_select.argtypes = [vp, i32, i64, i32, vp, i32, vp, vp, vp, i32, i32, i64, i32, vp,
+                                         vp, vp, vp, sz, vp, vp]
+        lib.rvq_shard_apply.argtypes = [vp, i32, i64, i32, vp, i32, ctypes.POINTER(vp), i32,
+                                        ctypes.POINTER(i32), i32, i32, vp, vp, vp, sz, vp, vp]
+        lib.rvq_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
+        lib.rvq_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
+        lib.rvq_ipc_close.argtypes = [vp, sz]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
                    "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc",
                    "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
-                   "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences"):
+                   "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
+                   "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply", "rvq_ipc_export",
+                   "rvq_ipc_import", "rvq_ipc_close"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -201,6 +214,53 @@ def rvq_balance_sequences(lengths, world):
 def rvq_gather_sequences(cache_ids, L, cache_offsets, S, select, M, out_offsets, out_ids, status=None, stream=None):
     return load().rvq_gather_sequences(_ptr(cache_ids), int(L), _ptr(cache_offsets), int(S), _ptr(select), int(M),
                                        _ptr(out_offsets), _ptr(out_ids), _ptr(status), _stream(stream))
+
+
+def rvq_shard_workspace_size(N, D, K_shard):
+    out = ctypes.c_size_t(0)
+    code = load().rvq_shard_workspace_size(N, D, K_shard, ctypes.byref(out))
+    return code, out.value
+
+
+def rvq_shard_select(features, f_dtype, N, D, shard_codebooks, cb_dtype, shard_operand, shard_norms, shard_stats,
+                     L, K_shard, k0, l, residual, sel, fallbacks, workspace, workspace_bytes, status=None,
+                     stream=None):
+    return load().rvq_shard_select(_ptr(features), f_dtype, N, D, _ptr(shard_codebooks), cb_dtype,
+                                   _ptr(shard_operand), _ptr(shard_norms), _ptr(shard_stats), L, K_shard, k0, l,
+                                   _ptr(residual), _ptr(sel), _ptr(fallbacks), _ptr(workspace), workspace_bytes,
+                                   _ptr(status), _stream(stream))
+
+
+def rvq_shard_apply(features, f_dtype, N, D, sel_all, W, shard_codebooks, cb_dtype, shard_K, L, l, ids, residual,
+                    workspace, workspace_bytes, status=None, stream=None):
+    """shard_codebooks: W device pointers (ints or tensors); shard_K: W codeword counts (host)."""
+    ptrs = (ctypes.c_void_p * max(W, 1))(*[_ptr(p) for p in shard_codebooks])
+    ks = (ctypes.c_int * max(W, 1))(*[int(k) for k in shard_K])
+    return load().rvq_shard_apply(_ptr(features), f_dtype, N, D, _ptr(sel_all), W, ptrs, cb_dtype, ks, L, l,
+                                  _ptr(ids), _ptr(residual), _ptr(workspace), workspace_bytes, _ptr(status),
+                                  _stream(stream))
+
+
+def rvq_ipc_export(ptr):
+    """-> (status, handle bytes, offset) of the device allocation holding ptr."""
+    h = ctypes.create_string_buffer(RVQ_IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t(0)
+    code = load().rvq_ipc_export(_ptr(ptr), h, ctypes.byref(off))
+    return code, h.raw, off.value
+
+
+def rvq_ipc_import(handle, offset):
+    """-> (status, device pointer as int) mapping another process's allocation."""
+    if len(handle) != RVQ_IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be RVQ_IPC_HANDLE_BYTES bytes")
+    h = ctypes.create_string_buffer(bytes(handle), RVQ_IPC_HANDLE_BYTES)
+    out = ctypes.c_void_p(None)
+    code = load().rvq_ipc_import(h, int(offset), ctypes.byref(out))
+    return code, (out.value or 0)
+
+
+def rvq_ipc_close(ptr, offset):
+    return load().rvq_ipc_close(_ptr(ptr), int(offset))
 
 
 def rvq_selftest_wait_timeout(counter, status, limit_us, stream=None):

@@ -2147,6 +2147,13 @@ struct Layout {
   size_t R, Rt, rowstat, cand, fb_list, fb_count, sync, sync_end, ex_part, total;
 };
 
+// The row state (fp32 residual, its bf16 operand copy, row statistics) opens every workspace;
+// its size depends on N and D only.
+inline size_t row_state_bytes(int64_t N, int D) {
+  return align256(static_cast<size_t>(N) * D * 4) + align256(static_cast<size_t>(N) * D * 2) +
+         align256(static_cast<size_t>(N) * 8);
+}
+
 inline Layout make_layout(int64_t N, int D, const Plan &p) {
   Layout w;
   size_t off = 0;
@@ -2156,7 +2163,7 @@ inline Layout make_layout(int64_t N, int D, const Plan &p) {
   off += align256(static_cast<size_t>(N) * D * 2);
   w.rowstat = off;
   off += align256(static_cast<size_t>(N) * 8);
-  w.cand = off;
+  w.cand = off;  // == row_state_bytes(N, D)
   off += align256(static_cast<size_t>(p.RT) * p.maxs * BM * TOPK * 8);
   w.fb_list = off;
   off += align256(static_cast<size_t>(N) * 4);
@@ -2660,4 +2667,494 @@ extern "C" int rvq_encode_noalloc(const void *features, int f_dtype, int64_t N, 
   if (st != RVQ_OK) return st;
   return rvq_encode(features, f_dtype, N, D, codebooks, cb_dtype, cb_operand, norms, level_stats, L, K, offsets, B,
                     ids, residual, recon, fallbacks, scratch, RVQ_NOALLOC_SCRATCH_BYTES, status, stream);
+}
+
+// ---------------------------------------------------------------- codebook-sharded encode
+//
+// The codebook axis split over W ranks: rank w holds codewords [k0_w, k0_w + K_w) of every level
+// (k0_w = K_0 + ... + K_{w-1}) and all N rows.  Per level:
+//   select (each rank): the distance GEMM over the shard, then shard_select_kernel certifies each
+//     row's candidates and rescans them exactly, writing the shard's nearest codeword with its
+//     exact distance ||r - c||^2; rows the certificate cannot settle get an exact scan of the
+//     shard (shard_fallback_kernel).
+//   exchange (caller): every rank gathers the W per-rank arrays.
+//   apply (each rank): shard_apply_kernel takes the lowest (distance, id) pair of each row, reads
+//     that codeword from its owner's shard (a peer pointer when the owner is another GPU) and
+//     updates the replicated residual exactly like the single-GPU path, so the replicas stay
+//     bit-identical.
+// The nearest codeword over all K is the nearest among the shards' nearest ones (ties to the
+// lowest id, which is also the lowest rank), so the ids are those of the one-GPU encode.
+namespace rvq {
+namespace enc {
+
+// One lane's share of ||r - c||^2 with every rounding explicit (no contraction), so that all
+// callers get bit-identical distances for equal rows: equal codewords held by different shards
+// tie exactly and go to the lowest id.
+template <int NCH>
+__device__ __forceinline__ double lane_sq_dist(const float4 (&rv)[NCH], const float4 (&c)[NCH]) {
+  double s = 0.0;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const double e0 = static_cast<double>(rv[k].x) - c[k].x, e1 = static_cast<double>(rv[k].y) - c[k].y;
+    const double e2 = static_cast<double>(rv[k].z) - c[k].z, e3 = static_cast<double>(rv[k].w) - c[k].w;
+    const double q = __dadd_rn(__dadd_rn(__dadd_rn(__dmul_rn(e0, e0), __dmul_rn(e1, e1)), __dmul_rn(e2, e2)),
+                               __dmul_rn(e3, e3));
+    s = __dadd_rn(s, q);
+  }
+  return s;
+}
+
+template <int SRC, int NCH>
+__device__ __forceinline__ void load_row(const RowArgs &a, int64_t n, float4 (&rv)[NCH], int lane) {
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    rv[k] = i < a.D ? ld_src4<SRC>(a.src, n * a.D + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <bool CB_BF16, int NCH>
+__device__ __forceinline__ void load_codeword(const void *cb, int64_t coff, int D, float4 (&c)[NCH], int lane) {
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int i = lane * 4 + k * 128;
+    c[k] = i < D ? ld4<CB_BF16>(cb, coff + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Nearest codeword of this shard for row n and its exact distance (one warp), from the shard's
+// candidate lists: same certificate as rescore_row, but the winner is always rescored exactly
+// because its distance is compared with the other shards'.  Uncertified rows are queued.
+template <bool CB_BF16, int SRC, int NCH>
+__device__ __forceinline__ void shard_best_row(const RowArgs &a, int64_t k0, double2 *sel, int64_t n, int lane) {
+  const int64_t rt = n / BM;
+  const int rin = static_cast<int>(n - rt * BM);
+  const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;
+  const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
+  const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
+  const int ncand = (c1 - c0 + 1) * TOPK;
+
+  float4 rv[NCH];
+  load_row<SRC, NCH>(a, n, rv, lane);
+  float dv[CPL];
+  int iv[CPL];
+#pragma unroll
+  for (int h = 0; h < CPL; ++h) {
+    const int e = lane + 32 * h;
+    dv[h] = inf_f();
+    iv[h] = -1;
+    if (e < ncand) {
+      const int slot = e / TOPK, t = e - slot * TOPK;
+      const float2 c = __ldcg(a.cand + ((rt * a.maxs + slot) * BM + rin) * TOPK + t);
+      dv[h] = c.x;
+      iv[h] = __float_as_int(c.y);
+    }
+  }
+  float2 rs = make_float2(0.f, 0.f);
+  if constexpr (SRC == SRC_X_BF16) {
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) q += rv[k].x * rv[k].x + rv[k].y * rv[k].y + rv[k].z * rv[k].z + rv[k].w * rv[k].w;
+    rs = make_float2(0.f, __fsqrt_ru(1.0001f * warp_sum_f(q)));
+  } else {
+    rs = __ldcg(a.rowstat + n);
+  }
+
+  float tl = inf_f(), ml = inf_f();
+#pragma unroll
+  for (int h = 0; h < CPL; ++h) {
+    const int e = lane + 32 * h;
+    if (e < ncand && (e % TOPK) == TOPK - 1) tl = fminf(tl, dv[h]);
+    ml = fminf(ml, dv[h]);
+  }
+  const float T = warp_min_f(tl);
+  const float dmin = warp_min_f(ml);
+  const float E = error_bound(a.stats, rs, a.D) + 7.62939453125e-06f * (fabsf(dmin) + (T < 1e30f ? fabsf(T) : 0.f));
+  const float lim = dmin + 2.f * E;
+
+  double rr = 0.0;
+#pragma unroll
+  for (int k = 0; k < NCH; ++k)
+    rr += static_cast<double>(rv[k].x) * rv[k].x + static_cast<double>(rv[k].y) * rv[k].y +
+          static_cast<double>(rv[k].z) * rv[k].z + static_cast<double>(rv[k].w) * rv[k].w;
+  rr = warp_sum_d(rr);
+  double best = inf_d();
+  int best_id = 0x7fffffff;
+#pragma unroll
+  for (int h = 0; h < CPL; ++h) {
+    unsigned mask = __ballot_sync(0xffffffffu, iv[h] >= 0 && dv[h] <= lim);
+    while (mask) {
+      const int srcl = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const int id = __shfl_sync(0xffffffffu, iv[h], srcl);
+      float4 c[NCH];
+      load_codeword<CB_BF16, NCH>(a.cb, (static_cast<int64_t>(a.l) * a.K + id) * a.D, a.D, c, lane);
+      const double dd = warp_sum_d(lane_sq_dist<NCH>(rv, c));
+      if (dd < best || (dd == best && id < best_id)) {
+        best = dd;
+        best_id = id;
+      }
+    }
+  }
+  const bool certified = best_id != 0x7fffffff && (best - rr) < (static_cast<double>(T) - static_cast<double>(E));
+  if (!certified) {
+    if (lane == 0) {
+      const int pos = atomicAdd(a.fb_count, 1);
+      a.fb_list[pos] = static_cast<int32_t>(n);
+    }
+    return;
+  }
+  if (lane == 0) sel[n] = make_double2(best, static_cast<double>(k0 + best_id));
+}
+
+template <bool CB_BF16, int SRC, int NCH>
+__global__ void __launch_bounds__(256, 2) shard_select_kernel(const RowArgs a, int64_t k0, double2 *sel) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (n >= a.N) return;
+  shard_best_row<CB_BF16, SRC, NCH>(a, k0, sel, n, threadIdx.x & 31);
+}
+
+// Exact scan of the shard's K codewords for each queued row (the block's 8 warps split the
+// codewords; every warp keeps the row in registers).  Writes (distance, global id), or (+inf, -1)
+// when no distance compares (non-finite inputs).
+template <bool CB_BF16, int SRC, int NCH>
+__global__ void __launch_bounds__(256) shard_fallback_kernel(const RowArgs a, int64_t k0, double2 *sel) {
+  constexpr int NW = 8;
+  __shared__ double wbest[NW];
+  __shared__ int wid[NW];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int count = *a.fb_count;
+  for (int j = blockIdx.x; j < count; j += gridDim.x) {
+    const int64_t n = a.fb_list[j];
+    float4 rv[NCH];
+    load_row<SRC, NCH>(a, n, rv, lane);
+    double bd = inf_d();
+    int bk = 0x7fffffff;
+    for (int k = warp; k < a.K; k += NW) {
+      float4 c[NCH];
+      load_codeword<CB_BF16, NCH>(a.cb, (static_cast<int64_t>(a.l) * a.K + k) * a.D, a.D, c, lane);
+      const double d = warp_sum_d(lane_sq_dist<NCH>(rv, c));
+      if (d < bd) {  // k ascends within a warp: the first of equal distances stays
+        bd = d;
+        bk = k;
+      }
+    }
+    if (lane == 0) {
+      wbest[warp] = bd;
+      wid[warp] = bk;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double b = wbest[0];
+      int k = wid[0];
+      for (int w = 1; w < NW; ++w)
+        if (wbest[w] < b || (wbest[w] == b && wid[w] < k)) {
+          b = wbest[w];
+          k = wid[w];
+        }
+      sel[n] = k == 0x7fffffff ? make_double2(inf_d(), -1.0) : make_double2(b, static_cast<double>(k0 + k));
+    }
+    __syncthreads();  // wbest is rewritten by the next row
+  }
+}
+
+struct ShardApplyArgs {
+  const double2 *sel;  // [W, N]: each rank's (exact distance, global id) per row
+  int W;
+  const void *cb[RVQ_MAX_SHARDS];  // rank w's stored codebooks [L, Kw[w], D] (peer pointers allowed)
+  int Kw[RVQ_MAX_SHARDS];
+  int64_t k0[RVQ_MAX_SHARDS];
+};
+
+// Overall nearest codeword of row n (lowest distance, then lowest id) and the residual update.
+template <bool CB_BF16, int SRC, int NCH>
+__global__ void __launch_bounds__(256, 2) shard_apply_kernel(const RowArgs a, const ShardApplyArgs s) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (n >= a.N) return;
+  double b = inf_d();
+  int id = 0x7fffffff, w = -1;
+  if (lane < s.W) {
+    const double2 v = __ldcg(s.sel + static_cast<int64_t>(lane) * a.N + n);
+    const double lo = static_cast<double>(s.k0[lane]);
+    if (v.x == v.x && v.y >= lo && v.y < lo + static_cast<double>(s.Kw[lane])) {
+      b = v.x;
+      id = static_cast<int>(v.y);
+      w = lane;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, b, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, id, off);
+    const int ow = __shfl_xor_sync(0xffffffffu, w, off);
+    if (ow >= 0 && (w < 0 || ob < b || (ob == b && oi < id))) {
+      b = ob;
+      id = oi;
+      w = ow;
+    }
+  }
+  if (w < 0) {  // no rank produced a usable pair: only reachable with non-finite inputs
+    if (lane == 0) {
+      a.ids[n * a.L + a.l] = -1;
+      set_status(a.status, RVQ_ERR_ARG);
+    }
+    return;
+  }
+  float4 rv[NCH], c[NCH];
+  load_row<SRC, NCH>(a, n, rv, lane);
+  load_codeword<CB_BF16, NCH>(s.cb[w], (static_cast<int64_t>(a.l) * s.Kw[w] + (id - s.k0[w])) * a.D, a.D, c, lane);
+  apply_row<NCH>(a, n, rv, c, id, lane);
+}
+
+inline Plan make_shard_plan(int64_t N, int Ks, int D, int sms) {
+  Plan p = make_plan(N, Ks, D, 1, sms);
+  p.flow = false;  // one level per call: the per-level distance kernel
+  return p;
+}
+
+template <bool CB_BF16, int SRC>
+inline cudaError_t launch_shard_select(const RowArgs &ra, int64_t k0, double2 *sel, int nch, unsigned row_blocks,
+                                       unsigned fb_blocks, cudaStream_t s) {
+  cudaError_t e;
+  switch (nch) {
+    case 1:
+      e = launch_pdl(shard_select_kernel<CB_BF16, SRC, 1>, dim3(row_blocks), dim3(256), 0, s, ra, k0, sel);
+      if (e == cudaSuccess)
+        e = launch_pdl(shard_fallback_kernel<CB_BF16, SRC, 1>, dim3(fb_blocks), dim3(256), 0, s, ra, k0, sel);
+      return e;
+    case 2:
+      e = launch_pdl(shard_select_kernel<CB_BF16, SRC, 2>, dim3(row_blocks), dim3(256), 0, s, ra, k0, sel);
+      if (e == cudaSuccess)
+        e = launch_pdl(shard_fallback_kernel<CB_BF16, SRC, 2>, dim3(fb_blocks), dim3(256), 0, s, ra, k0, sel);
+      return e;
+    case 4:
+      e = launch_pdl(shard_select_kernel<CB_BF16, SRC, 4>, dim3(row_blocks), dim3(256), 0, s, ra, k0, sel);
+      if (e == cudaSuccess)
+        e = launch_pdl(shard_fallback_kernel<CB_BF16, SRC, 4>, dim3(fb_blocks), dim3(256), 0, s, ra, k0, sel);
+      return e;
+    default:
+      e = launch_pdl(shard_select_kernel<CB_BF16, SRC, 8>, dim3(row_blocks), dim3(256), 0, s, ra, k0, sel);
+      if (e == cudaSuccess)
+        e = launch_pdl(shard_fallback_kernel<CB_BF16, SRC, 8>, dim3(fb_blocks), dim3(256), 0, s, ra, k0, sel);
+      return e;
+  }
+}
+
+template <bool CB_BF16, int SRC>
+inline cudaError_t launch_shard_apply(const RowArgs &ra, const ShardApplyArgs &sa, int nch, unsigned row_blocks,
+                                      cudaStream_t s) {
+  switch (nch) {
+    case 1: return launch_pdl(shard_apply_kernel<CB_BF16, SRC, 1>, dim3(row_blocks), dim3(256), 0, s, ra, sa);
+    case 2: return launch_pdl(shard_apply_kernel<CB_BF16, SRC, 2>, dim3(row_blocks), dim3(256), 0, s, ra, sa);
+    case 4: return launch_pdl(shard_apply_kernel<CB_BF16, SRC, 4>, dim3(row_blocks), dim3(256), 0, s, ra, sa);
+    default: return launch_pdl(shard_apply_kernel<CB_BF16, SRC, 8>, dim3(row_blocks), dim3(256), 0, s, ra, sa);
+  }
+}
+
+// Feature widths of the sharded path: the register-resident row kernels.
+inline bool shard_width_ok(int D) { return D >= 64 && D <= 1024 && D % 64 == 0; }
+
+}  // namespace enc
+}  // namespace rvq
+
+extern "C" int rvq_shard_workspace_size(int64_t N, int D, int K_shard, size_t *bytes) {
+  using namespace rvq;
+  if (!bytes || N < 0 || D < 1 || K_shard < 1) return RVQ_ERR_ARG;
+  if (!enc::shard_width_ok(D) || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  int sms = 0;
+  const int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const enc::Plan p = enc::make_shard_plan(std::max<int64_t>(N, 1), K_shard, D, sms);
+  *bytes = enc::make_layout(N, D, p).total;
+  return RVQ_OK;
+}
+
+extern "C" int rvq_shard_select(const void *features, int f_dtype, int64_t N, int D, const void *shard_codebooks,
+                                int cb_dtype, const void *shard_operand, const float *shard_norms,
+                                const float *shard_stats, int L, int K_shard, int64_t k0, int l, float *residual,
+                                double *sel, int32_t *fallbacks, void *workspace, size_t workspace_bytes,
+                                int32_t *status, void *stream) {
+  using namespace rvq;
+  using namespace rvq::enc;
+  if (N < 0 || D < 1 || L < 1 || K_shard < 1 || k0 < 0 || l < 0 || l >= L) return RVQ_ERR_ARG;
+  if ((f_dtype != RVQ_F32 && f_dtype != RVQ_BF16) || (cb_dtype != RVQ_F32 && cb_dtype != RVQ_BF16))
+    return RVQ_ERR_ARG;
+  if (!shard_width_ok(D) || L > 64 || N >= (int64_t(1) << 31) || k0 + K_shard >= (int64_t(1) << 31))
+    return RVQ_ERR_UNSUPPORTED;
+  if (N == 0) return RVQ_OK;
+  if (!features || !shard_codebooks || !shard_norms || !shard_stats || !sel) return RVQ_ERR_ARG;
+  if (cb_dtype == RVQ_F32 && !shard_operand) return RVQ_ERR_ARG;
+  const void *op = cb_dtype == RVQ_BF16 ? shard_codebooks : shard_operand;
+  if (!aligned16(features) || !aligned16(shard_codebooks) || !aligned16(op) || !aligned16(shard_norms) ||
+      !aligned16(sel) || (residual && !aligned16(residual)))
+    return RVQ_ERR_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RVQ_ERR_WORKSPACE;
+  int sms = 0;
+  int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const Plan p = make_shard_plan(N, K_shard, D, sms);
+  const Layout w = make_layout(N, D, p);
+  if (workspace_bytes < w.total) return RVQ_ERR_WORKSPACE;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *R = residual ? residual : reinterpret_cast<float *>(ws + w.R);
+  __nv_bfloat16 *Rt = reinterpret_cast<__nv_bfloat16 *>(ws + w.Rt);
+  float2 *rowstat = reinterpret_cast<float2 *>(ws + w.rowstat);
+  float2 *cand = reinterpret_cast<float2 *>(ws + w.cand);
+  int32_t *fb_list = reinterpret_cast<int32_t *>(ws + w.fb_list);
+  int32_t *fb_count = reinterpret_cast<int32_t *>(ws + w.fb_count);
+
+  // Level 0 scores the features: bf16 features are their own operand; fp32 features get a bf16
+  // copy and row statistics first.  Later levels score the residual operand written by apply.
+  const bool x_is_operand = l == 0 && f_dtype == RVQ_BF16;
+  const int64_t row_blocks = (N * 32 + 255) / 256;
+  if (l == 0 && !x_is_operand) {
+    const cudaError_t e = launch_pdl(init_kernel<false, false>, dim3(static_cast<unsigned>(row_blocks)), dim3(256), 0,
+                                     s, features, N, D, R, Rt, rowstat, fb_count, 0,
+                                     static_cast<const int64_t *>(nullptr), int64_t(0), status);
+    note_launch();
+    if (e != cudaSuccess) return RVQ_ERR_CUDA;
+  }
+  CUtensorMap tmA, tmB;
+  if (!make_map(&tmA, x_is_operand ? features : static_cast<const void *>(Rt), N, D, BM)) return RVQ_ERR_CUDA;
+  if (!make_map(&tmB, static_cast<const uint8_t *>(op) + static_cast<size_t>(l) * K_shard * D * 2, K_shard, D,
+                p.pair ? BN / 2 : BN))
+    return RVQ_ERR_CUDA;
+  const int epi = epilogue_warps(D);
+  if (!gemm_attrs_ready(epi)) return RVQ_ERR_CUDA;
+  GemmArgs ga;
+  ga.norms = shard_norms + static_cast<size_t>(l) * K_shard;
+  ga.N = N;
+  ga.K = K_shard;
+  ga.D = D;
+  ga.U = p.U;
+  ga.Tc = p.Tc;
+  ga.G = p.G;
+  ga.maxs = p.maxs;
+  ga.cand = cand;
+  ga.status = status;
+  ga.zero_counter = fb_count;  // this call's count of exact shard scans
+  profile_begin(s);
+  const cudaError_t ge = launch_gemm(epi, p.pair, p.G, s, tmA, tmB, ga);
+  profile_end(s);
+  note_launch();
+  if (ge != cudaSuccess) return RVQ_ERR_CUDA;
+
+  RowArgs ra;
+  ra.N = N;
+  ra.D = D;
+  ra.K = K_shard;
+  ra.L = L;
+  ra.l = l;
+  ra.Tc = p.Tc;
+  ra.G = p.G;
+  ra.maxs = p.maxs;
+  ra.pair = p.pair ? 1 : 0;
+  ra.U = p.U;
+  ra.rt0 = 0;
+  ra.nslots = 0;
+  ra.cand = cand;
+  ra.rowstat = rowstat;
+  ra.R = R;
+  ra.Rt = Rt;
+  ra.cb = shard_codebooks;
+  ra.stats = shard_stats + static_cast<size_t>(l) * RVQ_LEVEL_STATS;
+  ra.ids = nullptr;
+  ra.fb_list = fb_list;
+  ra.fb_count = fb_count;
+  ra.status = status;
+  ra.last = l == L - 1;
+  ra.src = l == 0 ? features : static_cast<const void *>(R);
+  ra.fb_next = nullptr;
+  ra.offsets = nullptr;
+  ra.B = 0;
+  double2 *sel2 = reinterpret_cast<double2 *>(sel);
+  const int nch = row_chunks(D);
+  const unsigned rb = static_cast<unsigned>(row_blocks), fb = static_cast<unsigned>(2 * sms);
+  const bool cbb = cb_dtype == RVQ_BF16;
+  cudaError_t e;
+  if (l > 0)
+    e = cbb ? launch_shard_select<true, SRC_R>(ra, k0, sel2, nch, rb, fb, s)
+            : launch_shard_select<false, SRC_R>(ra, k0, sel2, nch, rb, fb, s);
+  else if (f_dtype == RVQ_BF16)
+    e = cbb ? launch_shard_select<true, SRC_X_BF16>(ra, k0, sel2, nch, rb, fb, s)
+            : launch_shard_select<false, SRC_X_BF16>(ra, k0, sel2, nch, rb, fb, s);
+  else
+    e = cbb ? launch_shard_select<true, SRC_X_F32>(ra, k0, sel2, nch, rb, fb, s)
+            : launch_shard_select<false, SRC_X_F32>(ra, k0, sel2, nch, rb, fb, s);
+  note_launch(2);
+  if (e != cudaSuccess) return RVQ_ERR_CUDA;
+  if (fallbacks && cudaMemcpyAsync(fallbacks + l, fb_count, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return RVQ_ERR_CUDA;
+  return RVQ_OK;
+}
+
+extern "C" int rvq_shard_apply(const void *features, int f_dtype, int64_t N, int D, const double *sel_all, int W,
+                               const void *const *shard_codebooks, int cb_dtype, const int *shard_K, int L, int l,
+                               int32_t *ids, float *residual, void *workspace, size_t workspace_bytes,
+                               int32_t *status, void *stream) {
+  using namespace rvq;
+  using namespace rvq::enc;
+  if (N < 0 || D < 1 || L < 1 || l < 0 || l >= L || W < 1) return RVQ_ERR_ARG;
+  if ((f_dtype != RVQ_F32 && f_dtype != RVQ_BF16) || (cb_dtype != RVQ_F32 && cb_dtype != RVQ_BF16))
+    return RVQ_ERR_ARG;
+  if (!shard_width_ok(D) || L > 64 || N >= (int64_t(1) << 31) || W > RVQ_MAX_SHARDS) return RVQ_ERR_UNSUPPORTED;
+  if (!shard_codebooks || !shard_K) return RVQ_ERR_ARG;
+  ShardApplyArgs sa = {};
+  int64_t k = 0;
+  for (int r = 0; r < W; ++r) {
+    if (!shard_codebooks[r] || !aligned16(shard_codebooks[r]) || shard_K[r] < 1) return RVQ_ERR_ARG;
+    sa.cb[r] = shard_codebooks[r];
+    sa.Kw[r] = shard_K[r];
+    sa.k0[r] = k;
+    k += shard_K[r];
+  }
+  if (k >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  if (N == 0) return RVQ_OK;
+  if (!features || !sel_all || !ids || !aligned16(features) || !aligned16(sel_all) ||
+      (residual && !aligned16(residual)) || (reinterpret_cast<uintptr_t>(ids) & 3u))
+    return RVQ_ERR_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RVQ_ERR_WORKSPACE;
+  if (workspace_bytes < row_state_bytes(N, D)) return RVQ_ERR_WORKSPACE;
+  sa.sel = reinterpret_cast<const double2 *>(sel_all);
+  sa.W = W;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  RowArgs ra = {};
+  ra.N = N;
+  ra.D = D;
+  ra.K = static_cast<int>(k);
+  ra.L = L;
+  ra.l = l;
+  ra.R = residual ? residual : reinterpret_cast<float *>(ws);
+  ra.Rt = reinterpret_cast<__nv_bfloat16 *>(ws + align256(static_cast<size_t>(N) * D * 4));
+  ra.rowstat = reinterpret_cast<float2 *>(ws + align256(static_cast<size_t>(N) * D * 4) +
+                                          align256(static_cast<size_t>(N) * D * 2));
+  ra.ids = ids;
+  ra.status = status;
+  ra.last = l == L - 1;
+  ra.src = l == 0 ? features : static_cast<const void *>(ra.R);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nch = row_chunks(D);
+  const unsigned rb = static_cast<unsigned>((N * 32 + 255) / 256);
+  const bool cbb = cb_dtype == RVQ_BF16;
+  cudaError_t e;
+  if (l > 0)
+    e = cbb ? launch_shard_apply<true, SRC_R>(ra, sa, nch, rb, s) : launch_shard_apply<false, SRC_R>(ra, sa, nch, rb, s);
+  else if (f_dtype == RVQ_BF16)
+    e = cbb ? launch_shard_apply<true, SRC_X_BF16>(ra, sa, nch, rb, s)
+            : launch_shard_apply<false, SRC_X_BF16>(ra, sa, nch, rb, s);
+  else
+    e = cbb ? launch_shard_apply<true, SRC_X_F32>(ra, sa, nch, rb, s)
+            : launch_shard_apply<false, SRC_X_F32>(ra, sa, nch, rb, s);
+  note_launch();
+  return e == cudaSuccess ? RVQ_OK : RVQ_ERR_CUDA;
 }

@@ -90,6 +90,47 @@ def test_host_argument_checks(lib):
     assert L.rvq_gather_sequences(None, 8, 16, 1, 16, 1, 16, 16, None, None) == -1 # no cache
     assert L.rvq_selftest_wait_timeout(None, 16, 1000, None) == -1               # no counter
     assert L.rvq_selftest_wait_timeout(16, 16, 0, None) == -1                  # limit out of range
+    sz = ctypes.c_size_t(0)
+    assert L.rvq_shard_workspace_size(100, 1024, 4096, None) == -1             # no output
+    assert L.rvq_shard_workspace_size(100, 2048, 4096, ctypes.byref(sz)) == -2  # D > 1024
+    assert L.rvq_shard_workspace_size(100, 96, 4096, ctypes.byref(sz)) == -2   # D % 64
+    sel = L.rvq_shard_select
+    sargs = [16, 0, 0, 64, 16, 0, 16, 16, 16, 2, 8, 0, 0, None, 16, None, 256, 1 << 20, None, None]
+    assert sel(*sargs) == 0                                                    # N = 0: no-op
+    s1 = list(sargs); s1[12] = 2
+    assert sel(*s1) == -1                                                      # level l >= L
+    s2 = list(sargs); s2[2] = 5; s2[6] = None
+    assert sel(*s2) == -1                                                      # fp32 shard needs operand copy
+    s3 = list(sargs); s3[2] = 5; s3[3] = 2048
+    assert sel(*s3) == -2                                                      # D > 1024
+    s4 = list(sargs); s4[2] = 5; s4[16] = None
+    assert sel(*s4) == -3                                                      # no workspace
+    s5 = list(sargs); s5[2] = 5; s5[14] = 24
+    assert sel(*s5) == -1                                                      # misaligned sel
+    s6 = list(sargs); s6[11] = -1
+    assert sel(*s6) == -1                                                      # negative first id
+    app = L.rvq_shard_apply
+    vp2 = (ctypes.c_void_p * 2)(16, 32)
+    k2 = (ctypes.c_int * 2)(8, 8)
+    aargs = [16, 0, 0, 64, 16, 2, vp2, 0, k2, 2, 0, 16, None, 256, 1 << 20, None, None]
+    assert app(*aargs) == 0                                                    # N = 0: no-op
+    a1 = list(aargs); a1[5] = 0
+    assert app(*a1) == -1                                                      # no shards
+    a2 = list(aargs); a2[5] = 17
+    assert app(*a2) == -2                                                      # above RVQ_MAX_SHARDS
+    a3 = list(aargs); a3[8] = (ctypes.c_int * 2)(8, 0)
+    assert app(*a3) == -1                                                      # empty shard
+    a4 = list(aargs); a4[6] = (ctypes.c_void_p * 2)(16, 40)
+    assert app(*a4) == -1                                                      # misaligned peer pointer
+    a5 = list(aargs); a5[2] = 5; a5[14] = 100
+    assert app(*a5) == -3                                                      # workspace below the row state
+    a6 = list(aargs); a6[10] = 2
+    assert app(*a6) == -1                                                      # level l >= L
+    off = ctypes.c_size_t(0)
+    h = ctypes.create_string_buffer(mvt.RVQ_IPC_HANDLE_BYTES)
+    assert L.rvq_ipc_export(None, h, ctypes.byref(off)) == -1
+    assert L.rvq_ipc_import(None, 0, ctypes.byref(ctypes.c_void_p())) == -1
+    assert L.rvq_ipc_close(None, 0) == -1
 
 
 def test_missing_library_fails_loudly(tmp_path):
