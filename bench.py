@@ -444,25 +444,39 @@ def run_ours(args, rank, world, local_rank):
     embed = None
     if detok_only:
         gtab = torch.zeros((L, K, D), dtype=torch.float32, device=dev)
+        code, eb_ws_bytes = mvt.rvq_embed_backward_workspace_size(N, L, K, D)
+        check(code, "rvq_embed_backward_workspace_size")
+        eb_ws = torch.empty(eb_ws_bytes, dtype=torch.uint8, device=dev)
         ev2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        eb = []
-        for _ in range(min(args.steps + 2, 6)):
-            gtab.zero_()
-            flush_l2()
-            ev2[0].record(stream)
-            check(mvt.rvq_embed_backward(ids_in, N, L, K, D, rec2, gtab, status, stream), "rvq_embed_backward")
-            ev2[1].record(stream)
-            torch.cuda.synchronize(dev)
-            eb.append(ev2[0].elapsed_time(ev2[1]))
-        eb_ms = statistics.median(eb[1:]) if len(eb) > 1 else eb[0]
+
+        def time_backward(call):
+            t = []
+            for _ in range(min(args.steps + 2, 6)):
+                gtab.zero_()
+                flush_l2()
+                ev2[0].record(stream)
+                call()
+                ev2[1].record(stream)
+                torch.cuda.synchronize(dev)
+                t.append(ev2[0].elapsed_time(ev2[1]))
+            return statistics.median(t[1:]) if len(t) > 1 else t[0]
+
+        det_ms = time_backward(lambda: check(mvt.rvq_embed_backward_sorted(
+            ids_in, N, L, K, D, rec2, gtab, eb_ws, eb_ws_bytes, status, stream), "rvq_embed_backward_sorted"))
+        eb_ms = time_backward(lambda: check(mvt.rvq_embed_backward(ids_in, N, L, K, D, rec2, gtab, status, stream),
+                                            "rvq_embed_backward"))
         # algorithmic minimum: ids and g read once, every referenced gradient row read and written once
         used = sum(int(np.unique(g["planted"][:, l]).size) for l in range(L))
         eb_bytes = N * L * 4 + N * D * 4 + 2 * used * D * 4
+        hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
         embed = {"ms": eb_ms, "GB_per_s": eb_bytes / (eb_ms / 1e3) / 1e9, "algorithmic_bytes": eb_bytes,
-                 "frac_hbm": eb_bytes / (eb_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])),
+                 "frac_hbm": eb_bytes / (eb_ms / 1e3) / 1e9 / hbm,
                  "fp32x4_atomics_per_s": N * L * (D // 4) / (eb_ms / 1e3),
-                 "g": "decoded fp32 recon [N,D]", "kernel": "embed_backward_kernel"}
-        del gtab
+                 "kernel": "embed_backward_kernel (fp32x4 atomics)",
+                 "deterministic_ms": det_ms, "deterministic_frac_hbm": eb_bytes / (det_ms / 1e3) / 1e9 / hbm,
+                 "deterministic_kernels": "ss_hist/ss_prefix/ss_scan/ss_scatter (sort by id) + ss_sum + ss_fix",
+                 "g": "decoded fp32 recon [N,D]"}
+        del gtab, eb_ws
 
     # -------------------------------------------------- end to end through host buffers
     # Every step copies its features from pinned host memory and its ids + decoded recon back.

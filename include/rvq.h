@@ -179,6 +179,23 @@ RVQ_API int rvq_embed_backward(const int32_t *ids, int64_t N, int L, int K, int 
                                float *grad_tables, int32_t *status, void *stream);
 
 /*
+ * rvq_embed_backward_sorted -- the same table gradient as rvq_embed_backward, deterministic: the
+ * tokens of every level are sorted by id (a stable counting sort) and each gradient row receives
+ * its terms from one thread in an order fixed by the ids alone (ascending token index; ids with
+ * more than 256 tokens summed in pieces of 256 tokens, the pieces then added in ascending order),
+ * so repeated calls on the same inputs give bit-identical gradients.
+ * Each element still lies within (count - 1) * 2^-24 * sum of |terms| of the exact sum.
+ * workspace: >= rvq_embed_backward_workspace_size bytes of device memory, 256-byte aligned
+ * (RVQ_ERR_WORKSPACE otherwise); other arguments, status and id-range handling as in
+ * rvq_embed_backward.  Supported: N < 2^31, 1 <= L <= 64, 1 <= K <= 49151, H % 4 == 0.
+ * rvq_embed_backward_workspace_size writes the workspace bytes for these sizes into *bytes.
+ */
+RVQ_API int rvq_embed_backward_workspace_size(int64_t N, int L, int K, int H, size_t *bytes);
+RVQ_API int rvq_embed_backward_sorted(const int32_t *ids, int64_t N, int L, int K, int H, const float *grad_out,
+                                      float *grad_tables, void *workspace, size_t workspace_bytes,
+                                      int32_t *status, void *stream);
+
+/*
  * rvq_codebook_update -- one k-means (Lloyd) update of one codebook level: the step that fits the
  * fixed tokenizer whose ids the pages precompute offline (LongCat-2.5 technical blog, "Offline
  * Visual Preprocessing"; the pages do not describe the fitting: plain k-means on the level's input

@@ -30,7 +30,8 @@ EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_de
            "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
            "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
            "rvq_encode_noalloc", "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply",
-           "rvq_ipc_export", "rvq_ipc_import", "rvq_ipc_close")
+           "rvq_ipc_export", "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
+           "rvq_embed_backward_sorted")
 RVQ_MAX_SHARDS = 16
 RVQ_IPC_HANDLE_BYTES = 64
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -85,12 +86,15 @@ def load(path: str | None = None):
         lib.rvq_ipc_export.argtypes = [vp, vp, ctypes.POINTER(sz)]
         lib.rvq_ipc_import.argtypes = [vp, sz, ctypes.POINTER(vp)]
         lib.rvq_ipc_close.argtypes = [vp, sz]
+        lib.rvq_embed_backward_workspace_size.argtypes = [i64, i32, i32, i32, ctypes.POINTER(sz)]
+        lib.rvq_embed_backward_sorted.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, sz, vp, vp]
         for fn in ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_decode",
                    "rvq_profile_enable", "rvq_profile_read", "rvq_encode_noalloc",
                    "rvq_encode_levels_per_launch", "rvq_selftest_wait_timeout", "rvq_embed_backward",
                    "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
                    "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply", "rvq_ipc_export",
-                   "rvq_ipc_import", "rvq_ipc_close"):
+                   "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
+                   "rvq_embed_backward_sorted"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -193,6 +197,18 @@ def rvq_encode_levels_per_launch(N, D, L, K):
 def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stream=None):
     return load().rvq_embed_backward(_ptr(ids), int(N), int(L), int(K), int(H), _ptr(grad_out), _ptr(grad_tables),
                                      _ptr(status), _stream(stream))
+
+
+def rvq_embed_backward_workspace_size(N, L, K, H):
+    out = ctypes.c_size_t(0)
+    code = load().rvq_embed_backward_workspace_size(N, L, K, H, ctypes.byref(out))
+    return code, out.value
+
+
+def rvq_embed_backward_sorted(ids, N, L, K, H, grad_out, grad_tables, workspace, workspace_bytes, status=None,
+                              stream=None):
+    return load().rvq_embed_backward_sorted(_ptr(ids), N, L, K, H, _ptr(grad_out), _ptr(grad_tables),
+                                            _ptr(workspace), workspace_bytes, _ptr(status), _stream(stream))
 
 
 def rvq_codebook_update(points, ids, N, D, K, old_codebook, new_codebook, sums, counts, status=None, stream=None):

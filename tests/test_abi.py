@@ -131,6 +131,15 @@ def test_host_argument_checks(lib):
     assert L.rvq_ipc_export(None, h, ctypes.byref(off)) == -1
     assert L.rvq_ipc_import(None, 0, ctypes.byref(ctypes.c_void_p())) == -1
     assert L.rvq_ipc_close(None, 0) == -1
+    assert L.rvq_embed_backward_workspace_size(10, 2, 8, 16, None) == -1
+    assert L.rvq_embed_backward_workspace_size(10, 2, 49152, 16, ctypes.byref(sz)) == -2     # K too large
+    assert L.rvq_embed_backward_workspace_size(10, 2, 8, 18, ctypes.byref(sz)) == -2         # H % 4
+    assert L.rvq_embed_backward_workspace_size(10, 2, 8, 16, ctypes.byref(sz)) == 0 and sz.value > 0
+    ebs = L.rvq_embed_backward_sorted
+    assert ebs(16, 0, 2, 8, 16, 16, 16, None, 0, None, None) == 0                           # N = 0: no-op
+    assert ebs(None, 5, 2, 8, 16, 16, 16, 256, 1 << 20, None, None) == -1                   # no ids
+    assert ebs(16, 5, 2, 8, 16, 16, 16, None, 0, None, None) == -3                          # no workspace
+    assert ebs(16, 5, 2, 8, 16, 16, 16, 256, 100, None, None) == -3                         # too small
 
 
 def test_missing_library_fails_loudly(tmp_path):
