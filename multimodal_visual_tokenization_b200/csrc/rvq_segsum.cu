@@ -16,17 +16,17 @@
 //   4. ss_scatter_kernel  per (level, chunk), one warp: tokens in ascending n go to their slots
 //                         (ranks among equal ids from __match_any_sync), so each segment lists its
 //                         tokens in ascending n: a stable counting sort
-//   5. ss_sum_kernel      per (column slice of 16, level): every group of 4 lanes (float4 each) streams
-//                         the positions of one run in ascending order with SS_DEPTH rows in flight per
-//                         lane (16-byte cp.async copies into a shared-memory ring, so the depth costs
-//                         no registers), and adds each segment's sum into its gradient row with one
-//                         float4 atomic (the only write of that element, so no ordering question
-//                         arises); a hot id's pieces go to scratch rows instead
+//   5. ss_sum_kernel      per (column slice of 32, level): every group of 4 lanes (2 float4 each)
+//                         streams the positions of one run in ascending order with SS_DEPTH rows in
+//                         flight per lane (16-byte cp.async copies into a shared-memory ring, so the
+//                         depth costs no registers), and adds each segment's sum into its gradient
+//                         row with float4 atomics (the only write of those elements, so no ordering
+//                         question arises); a hot id's pieces go to scratch rows instead
 //   6. ss_fix_kernel      per hot id: its pieces summed in order and added into the gradient row
 // Every gradient element is written by one thread, with its terms added in an order fixed by the
-// ids alone, so the result is bit-identical from run to run.  The grid runs slice-major: while one
-// 16-column slice of g (N x 64 bytes, 64 MiB at N = 2^20) is summed for all levels it stays in L2,
-// so g is read from HBM about once and the gathers are L2 reads.
+// ids alone, so the result is bit-identical from run to run.  The grid runs slice-major, so the
+// 32-column slice of g being summed for all levels (N x 128 bytes, one line per row) is reused
+// from L2 while it stays there.
 #include <algorithm>
 
 #include "rvq_device.cuh"
@@ -36,13 +36,13 @@ namespace rvq {
 namespace ss {
 
 constexpr int SS_CH = 8192;    // tokens per histogram / scatter block
-constexpr int SS_COLS = 16;    // gradient columns per slice: 4 lanes x float4
+constexpr int SS_COLS = 32;    // gradient columns per slice: 4 lanes x 2 float4 (one 128-byte line of a row)
 constexpr int SS_HOT = 256;    // segments longer than this are summed in pieces of this size
 constexpr int SS_RUN = 256;    // a run of segments is cut where a segment starts in a new window
 constexpr int SS_WARPS = 8;    // warps per block of the sum and fix kernels
 constexpr int SS_UNITS = SS_WARPS * 8;  // runs or pieces per block of the sum kernel (8 per warp)
-constexpr int SS_DEPTH = 16;   // g rows in flight per lane (shared-memory ring of 16-byte copies)
-constexpr int SS_SUM_SMEM = SS_WARPS * 32 * SS_DEPTH * 16;
+constexpr int SS_DEPTH = 8;    // g rows in flight per lane (shared-memory ring of 2 x 16-byte copies)
+constexpr int SS_SUM_SMEM = SS_WARPS * 32 * SS_DEPTH * 32;
 constexpr int SCAN_THREADS = 1024;
 constexpr int MAX_K = 49151;   // K + 1 histogram counters in <= 192 KiB of shared memory
 
@@ -138,10 +138,15 @@ __global__ void __launch_bounds__(256) ss_prefix_kernel(const Args a) {
   if (k >= nk) return;
   int32_t *hist = a.hist + static_cast<int64_t>(l) * a.nch * nk + k;
   int r = 0;
-  for (int64_t c = 0; c < a.nch; ++c) {
-    const int o = hist[c * nk];
-    hist[c * nk] = r;
-    r += o;
+  for (int64_t c = 0; c < a.nch; c += 8) {  // eight chunks' counts in flight at a time
+    int o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = c + u < a.nch ? hist[(c + u) * nk] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c + u < a.nch) hist[(c + u) * nk] = r;
+      r += o[u];
+    }
   }
   a.start[static_cast<int64_t>(l) * nk + k] = r;
 }
@@ -296,8 +301,8 @@ __global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int
   const int64_t s = b / (a.L * per_level);
   const int l = static_cast<int>((b / per_level) % a.L);
   const int64_t ib = b % per_level;
-  const int col = static_cast<int>(s) * SS_COLS + (lane & 3) * 4;
-  const bool active = col < a.H;
+  const int col = static_cast<int>(s) * SS_COLS + (lane & 3) * 8;  // this lane: col .. col + 7
+  const bool act0 = col < a.H, act1 = col + 4 < a.H;
   const int unit = (threadIdx.x >> 2);  // 0 .. SS_UNITS-1
   const int32_t *perm = a.perm + static_cast<int64_t>(l) * a.N;
   const int32_t *nz_start = a.nz_start + static_cast<int64_t>(l) * (a.K + 2);
@@ -342,47 +347,60 @@ __global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int
   // the segment after the current one (runs only), loaded ahead of its use
   int nkey = i + 1 < i1 ? __ldg(nz_key + i + 1) : 0;
   int64_t ne = i + 1 < i1 ? __ldg(nz_start + i + 2) : 0;
-  // Ring of SS_DEPTH slots per lane: position p's 16 bytes land in slot p % SS_DEPTH, stored
-  // slot-major (slot, thread) so the lanes of a warp touch consecutive 16-byte words.  Copies are
+  // Ring of SS_DEPTH slots per lane: position p's 2 x 16 bytes land in slot p % SS_DEPTH, stored
+  // (slot, half, thread) so the lanes of a warp touch consecutive 16-byte words.  Copies are
   // committed four positions per group, so SS_DEPTH / 4 groups are in flight.
+  constexpr int PF = SS_DEPTH / 4;
+  constexpr int T = SS_WARPS * 32;
   extern __shared__ float4 ring_all[];
-  float4 *ring = ring_all + threadIdx.x;  // slot t at ring[t * SS_WARPS * 32]
+  float4 *ring = ring_all + threadIdx.x;  // half h of slot t at ring[(2 t + h) * T]
   const float *gcol = a.g + col;
   auto issue4 = [&](int64_t p, const int (&nidx)[4]) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (nidx[u] >= 0 && active)
-        cp_async16(ring + ((p + u) & (SS_DEPTH - 1)) * (SS_WARPS * 32), gcol + static_cast<int64_t>(nidx[u]) * a.H);
+    for (int u = 0; u < 4; ++u) {
+      const int t = static_cast<int>((p + u) & (SS_DEPTH - 1));
+      const float *src = gcol + static_cast<int64_t>(nidx[u]) * a.H;
+      if (nidx[u] >= 0 && act0) cp_async16(ring + (2 * t) * T, src);
+      if (nidx[u] >= 0 && act1) cp_async16(ring + (2 * t + 1) * T, src + 4);
+    }
     cp_async_commit();
   };
   auto perm4 = [&](int64_t p, int (&nidx)[4]) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) nidx[u] = p + u < j1 ? __ldg(perm + p + u) : -1;
   };
-  // token indices of the positions issued in the next four steps, four steps ahead (pn[q] holds
-  // positions j + SS_DEPTH + 4q .. during step q of a 16-position round)
-  static_assert(SS_DEPTH == 16, "the index ring below holds four steps of four positions");
-  int pn[4][4];
+  auto add4 = [](float4 &x, const float4 &y) {
+    x.x += y.x;
+    x.y += y.y;
+    x.z += y.z;
+    x.w += y.w;
+  };
+  // token indices of the positions issued in the next PF steps (pn[q] holds positions
+  // j + SS_DEPTH + 4q .. during step q of a round of 4 PF positions)
+  int pn[PF][4];
 #pragma unroll
-  for (int q = 0; q < SS_DEPTH / 4; ++q) {
+  for (int q = 0; q < PF; ++q) {
     perm4(j0 + 4 * q, pn[q]);
     issue4(j0 + 4 * q, pn[q]);
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) perm4(j0 + SS_DEPTH + 4 * q, pn[q]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t j16 = j0; j16 < j1; j16 += 16) {
+  for (int q = 0; q < PF; ++q) perm4(j0 + SS_DEPTH + 4 * q, pn[q]);
+  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+  for (int64_t jr = j0; jr < j1; jr += 4 * PF) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int64_t j = j16 + 4 * q;
+    for (int q = 0; q < PF; ++q) {
+      const int64_t j = jr + 4 * q;
       if (j < j1) {
-        cp_async_wait<SS_DEPTH / 4 - 1>();  // positions j .. j + 3 have landed
+        cp_async_wait<PF - 1>();  // positions j .. j + 3 have landed
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (j + u < j1) {
             if (j + u == e) {  // the previous segment of the run is complete: its only write
-              if (active) atomicAdd(reinterpret_cast<float4 *>(grad_l + static_cast<int64_t>(key) * a.H), acc);
-              acc = make_float4(0.f, 0.f, 0.f, 0.f);
+              float *d = grad_l + static_cast<int64_t>(key) * a.H;
+              if (act0) atomicAdd(reinterpret_cast<float4 *>(d), acc0);
+              if (act1) atomicAdd(reinterpret_cast<float4 *>(d + 4), acc1);
+              acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
+              acc1 = acc0;
               ++i;
               key = nkey;
               e = ne;
@@ -391,27 +409,27 @@ __global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int
                 ne = __ldg(nz_start + i + 2);
               }
             }
-            if (active) {
-              const float4 r = ring[((j + u) & (SS_DEPTH - 1)) * (SS_WARPS * 32)];
-              acc.x += r.x;
-              acc.y += r.y;
-              acc.z += r.z;
-              acc.w += r.w;
-            }
+            const int t = static_cast<int>((j + u) & (SS_DEPTH - 1));
+            if (act0) add4(acc0, ring[(2 * t) * T]);
+            if (act1) add4(acc1, ring[(2 * t + 1) * T]);
           }
         }
-        // the four slots just read (their values are already in acc) take positions j + SS_DEPTH ..
+        // the slots just read (their values are already in the sums) take positions j + SS_DEPTH ..
         issue4(j + SS_DEPTH, pn[q]);
-        perm4(j + SS_DEPTH + 16, pn[q]);
+        perm4(j + 2 * SS_DEPTH, pn[q]);
       }
     }
   }
   cp_async_wait<0>();
   if (j1 > j0) {
-    if (piece)
-      *reinterpret_cast<float4 *>(piece) = acc;  // padding columns of a piece row get zeros
-    else if (active)
-      atomicAdd(reinterpret_cast<float4 *>(grad_l + static_cast<int64_t>(key) * a.H), acc);
+    if (piece) {  // padding columns of a piece row get zeros
+      reinterpret_cast<float4 *>(piece)[0] = acc0;
+      reinterpret_cast<float4 *>(piece)[1] = acc1;
+    } else {
+      float *d = grad_l + static_cast<int64_t>(key) * a.H;
+      if (act0) atomicAdd(reinterpret_cast<float4 *>(d), acc0);
+      if (act1) atomicAdd(reinterpret_cast<float4 *>(d + 4), acc1);
+    }
   }
 }
 
