@@ -404,3 +404,53 @@ def test_cta_pair_kernel_matches_oracle():
     out = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True,
                          timeout=600)
     assert out.returncode == 0 and "pair ok" in out.stdout, out.stdout[-2000:] + out.stderr[-2000:]
+
+
+@pytest.mark.parametrize("N,L,K,D", [
+    (3001, 8, 500, 512),     # ragged token count, two 256-column slices
+    (1, 1, 7, 256),          # one token, one level (a gather of four rows, three of them padding)
+    (777, 3, 64, 768),       # L not a multiple of four
+    (4100, 16, 33, 256),     # the deepest level count the fixed decode handles
+])
+def test_bf16_decode_tma_gather_path(N, L, K, D):
+    """bf16 codebooks with D % 256 == 0 (in this process the register-gather kernel; the TMA gather
+    kernel in the subprocess test below): every row against the oracle, and an id outside [0, K)
+    sets the status and drops that level only."""
+    rng = np.random.Generator(np.random.PCG64([N, L, K, D]))
+    C = workloads.round_bf16(rng.standard_normal((L, K, D)).astype(np.float32))
+    ids = rng.integers(0, K, size=(N, L)).astype(np.int32)
+    tok = mvt.Tokenizer(dev(C, "bf16"))
+    rec = tok.decode(torch.from_numpy(ids).cuda())
+    torch.cuda.synchronize()
+    parity.check_recon(None, C, np.arange(N), ids, recon_gpu=rec.cpu().numpy())
+    bad = ids.copy()
+    bad[N // 2, L - 1] = K
+    bad[0, 0] = -1
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rec2 = tok.decode(torch.from_numpy(bad).cuda(), status=st, check=False).cpu().numpy()
+    assert int(st.item()) == -5
+    keep = (bad >= 0) & (bad < K)
+    for n in (0, N // 2):
+        want = sum(C[l, bad[n, l]].astype(np.float64) for l in range(L) if keep[n, l])
+        want = np.zeros(D) if isinstance(want, int) else want
+        assert np.allclose(rec2[n], want, rtol=1e-5, atol=1e-5)
+    others = np.ones(N, bool)
+    others[[0, N // 2]] = False
+    assert np.array_equal(rec2[others], rec.cpu().numpy()[others])
+
+
+def test_bf16_decode_tma_gather_kernel_in_subprocess():
+    """RVQ_DECODE_TMA=1 (fresh process): the same cases through the TMA gather decode kernel."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "from tests import test_gpu_parity as t\n"
+        "for case in [(3001, 8, 500, 512), (1, 1, 7, 256), (777, 3, 64, 768), (4100, 16, 33, 256)]:\n"
+        "    t.test_bf16_decode_tma_gather_path(*case)\n"
+        "print('tma decode ok')\n")
+    env = dict(os.environ, RVQ_DECODE_TMA="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0 and "tma decode ok" in out.stdout, out.stdout[-2000:] + out.stderr[-2000:]
