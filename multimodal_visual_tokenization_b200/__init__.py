@@ -10,6 +10,20 @@ library is missing.
 ``Tokenizer`` is the convenience layer a user calls: it holds a fixed codebook set with
 its prepared norms/operand copy (the pages' "fixed tokenizer"), and its ``encode`` /
 ``decode`` allocate outputs with torch and call the C entry points.
+
+Usage (one GPU)::
+
+    tok = Tokenizer(codebooks)                 # [L, K, D] float32 or bfloat16, on the GPU
+    ids, residual, recon = tok.encode(x, residual=True, recon=True)   # x [N, D]
+    feats = tok.decode(ids)                    # [N, D] float32 = sum_l C_l[ids[:, l]]
+
+Other entry points:
+* ``rvq_embed_backward`` (fp32 atomics) / ``rvq_embed_backward_sorted`` (bit-reproducible, with a
+  workspace): gradient of an embedding e[n] = sum_l E_l[ids[n, l]] with respect to its tables.
+* ``rvq_codebook_update``: one k-means step of a codebook level.
+* ``rvq_balance_sequences`` / ``rvq_gather_sequences``: packing id sequences for data-parallel
+  ranks.
+* ``sharded.ShardedTokenizer``: the codebook axis split over the ranks of a process group.
 """
 from __future__ import annotations
 
