@@ -19,8 +19,10 @@
  *
  * Conventions for every entry point
  *   - All array pointers are DEVICE pointers owned by the caller, 16-byte aligned,
- *     row-major and densely packed.  The library keeps no device memory between
- *     calls except lazily created profiling events.
+ *     row-major and densely packed.  The library allocates no device memory between
+ *     calls except lazily created profiling events.  It does hold one statically sized
+ *     array, the RVQ_NOALLOC_SCRATCH_BYTES (32 MiB) scratch of rvq_encode_noalloc, on every
+ *     device where librvq.so's module is loaded, whichever entry points the caller uses.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued
  *     asynchronously; the call returns after enqueueing.
  *   - The return value is an rvq_status.  Argument errors are detected on the host
@@ -133,7 +135,8 @@ RVQ_API int rvq_encode(const void *features, int f_dtype, int64_t N, int D,
  *   - Sizes whose rvq_encode_workspace_size exceeds RVQ_NOALLOC_SCRATCH_BYTES are rejected with
  *     RVQ_ERR_WORKSPACE before anything is enqueued (use rvq_encode with a workspace instead).
  *   - The first call on a device looks up the scratch array's device address with that device
- *     current (once per device); make that first call before any stream capture.
+ *     current (once per device, and again after the device's context was replaced, e.g. by
+ *     cudaDeviceReset); make that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents (the kernels
  *     initialise everything they read).  Calls that overlap on the GPU (different streams,
  *     or threads) race on it: serialise them.
@@ -316,11 +319,19 @@ RVQ_API int rvq_ipc_close(void *ptr, size_t offset);
  *   RVQ levels one bracketed launch covers (L when the all-levels kernel runs, else 1), so that a
  *   profiler can turn rvq_profile_read's totals into per-launch figures.  Same argument checks as
  *   rvq_encode_workspace_size.
+ * rvq_encode_candidate_layout: where an encode of this shape keeps its candidate lists in the
+ *   workspace, so that a test can read the approximate distances the tensor cores produced:
+ *   byte offset `*offset` of an array cand[ceil(N/128)][*slots][128][8] of 8-byte entries
+ *   (float d~, int32 id), one list of the 8 lowest d~ = fl(||c||^2) - 2 bf16(r).bf16(c) per
+ *   128-row tile, slot and row, written for the LAST level the call encoded (entries with
+ *   id < 0 are empty; slots a row tile does not use are left untouched).  Same argument checks
+ *   as rvq_encode_workspace_size.
  */
 RVQ_API int64_t rvq_launch_count(void);
 RVQ_API int rvq_profile_enable(int enable);
 RVQ_API int rvq_profile_read(int64_t *gemm_launches, double *gemm_ms);
 RVQ_API int rvq_encode_levels_per_launch(int64_t N, int D, int L, int K, int *levels);
+RVQ_API int rvq_encode_candidate_layout(int64_t N, int D, int L, int K, size_t *offset, int *slots);
 
 /*
  * Self-test of the bounded waits (no counterpart on the pages).  Every spin of the encode kernels

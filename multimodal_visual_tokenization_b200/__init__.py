@@ -45,7 +45,7 @@ EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_de
            "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
            "rvq_encode_noalloc", "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply",
            "rvq_ipc_export", "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
-           "rvq_embed_backward_sorted")
+           "rvq_embed_backward_sorted", "rvq_encode_candidate_layout")
 RVQ_MAX_SHARDS = 16
 RVQ_IPC_HANDLE_BYTES = 64
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -60,11 +60,10 @@ class RVQError(RuntimeError):
         self.code = code
 
 
-def load(path: str | None = None):
-    """Load librvq.so (built by `python -m multimodal_visual_tokenization_b200._build`).
-    RVQ_LIBRARY names another build of the same library (e.g. a tuning variant)."""
+def load():
+    """Load librvq.so (built in-tree by `python -m multimodal_visual_tokenization_b200._build`)."""
     global _lib
-    path = path or os.environ.get("RVQ_LIBRARY") or LIB_PATH
+    path = LIB_PATH
     with _lock:
         if _lib is not None:
             return _lib
@@ -87,6 +86,7 @@ def load(path: str | None = None):
         lib.rvq_profile_enable.argtypes = [i32]
         lib.rvq_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         lib.rvq_encode_levels_per_launch.argtypes = [i64, i32, i32, i32, ctypes.POINTER(i32)]
+        lib.rvq_encode_candidate_layout.argtypes = [i64, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(i32)]
         lib.rvq_selftest_wait_timeout.argtypes = [vp, vp, i64, vp]
         lib.rvq_embed_backward.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, vp]
         lib.rvq_codebook_update.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -108,7 +108,7 @@ def load(path: str | None = None):
                    "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
                    "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply", "rvq_ipc_export",
                    "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
-                   "rvq_embed_backward_sorted"):
+                   "rvq_embed_backward_sorted", "rvq_encode_candidate_layout"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -206,6 +206,14 @@ def rvq_encode_levels_per_launch(N, D, L, K):
     lv = ctypes.c_int32(0)
     code = load().rvq_encode_levels_per_launch(int(N), int(D), int(L), int(K), ctypes.byref(lv))
     return code, lv.value
+
+
+def rvq_encode_candidate_layout(N, D, L, K):
+    """-> (status, byte offset of the candidate lists in the encode workspace, slots per row tile)."""
+    off = ctypes.c_size_t(0)
+    slots = ctypes.c_int32(0)
+    code = load().rvq_encode_candidate_layout(int(N), int(D), int(L), int(K), ctypes.byref(off), ctypes.byref(slots))
+    return code, off.value, slots.value
 
 
 def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stream=None):

@@ -45,15 +45,15 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
-    """Compile librvq.so; `out`/`defines` build a variant elsewhere (tuning experiments)."""
-    target = out or LIB
-    if out is None and not force and not _stale():
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile librvq.so in-tree (skipped while it is newer than every source and header)."""
+    target = LIB
+    if not force and not _stale():
         return LIB
     nvcc = _nvcc()
     cuda_home = os.path.dirname(os.path.dirname(nvcc))
     tmp = target + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp,
+    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp,
            *sources(),
            "-Xlinker", f"-rpath,{os.path.join(cuda_home, 'lib64')}"]
     if verbose:

@@ -208,245 +208,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeBlocksPerSm) decode_
   if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
 }
 
-// ---------------------------------------------------------------- TMA gather decode (bf16)
-//
-// Optional path (RVQ_DECODE_TMA=1) for bf16 codebooks with D % 256 == 0 and L <= 16: the codeword
-// rows of a token are fetched by
-// the tensor memory accelerator (cp.async.bulk.tensor tile::gather4: four rows of one 256-column
-// slice per instruction) into a per-warp shared-memory ring, so every warp keeps kTmaDepth tokens'
-// rows in flight without holding them in registers.  Each warp is its own pipeline: lane 0 issues,
-// all 32 lanes wait on the stage's mbarrier, sum the rows (8 columns per lane, ascending level
-// order, fp32) and stream the result to recon.  An id outside [0, K) fetches row 0 of its level
-// and is left out of the sum.
-constexpr int kTmaWarps = 8;
-constexpr int kTmaCols = 256;           // columns per slice = the gather box width
-constexpr int kTmaRing = 24576;         // ring bytes per warp
-
-template <int LC>
-struct TmaCfg {
-  static constexpr int G4 = (LC + 3) / 4;                // gather4 loads per token
-  static constexpr int STAGE = G4 * 4 * kTmaCols * 2;    // bytes per token (padding rows fetch row 0)
-  static constexpr int DEPTH = kTmaRing / STAGE >= 2 ? kTmaRing / STAGE : 2;
-  static constexpr int WARP_BYTES = DEPTH * STAGE;
-  static constexpr int SMEM = kTmaWarps * WARP_BYTES + 1024;  // + alignment slack
-  static_assert(SMEM <= 232448, "decode ring above the per-block shared-memory limit");
-};
-
-__device__ __forceinline__ void tma_gather4(const CUtensorMap *m, uint64_t *bar, void *dst, int32_t x, int32_t r0,
-                                            int32_t r1, int32_t r2, int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
-template <int LC>
-__global__ void __launch_bounds__(kTmaWarps * 32, 1)
-    decode_tma_kernel(const __grid_constant__ CUtensorMap tm, const int32_t *__restrict__ ids, int64_t N, int K,
-                      int D, float *__restrict__ recon, int32_t *status) {
-  using C = TmaCfg<LC>;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full[kTmaWarps][C::DEPTH];
-  __shared__ int abort_flag;
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) abort_flag = 0;
-  if (lane == 0)
-    for (int s = 0; s < C::DEPTH; ++s) mbar_init(&full[warp][s], 1);
-  fence_mbar_init();
-  __syncthreads();
-  griddep_launch_dependents();
-  griddep_wait();
-  if (threadIdx.x == 0) tma_prefetch_desc(&tm);
-  uint8_t *ring = smem + warp * C::WARP_BYTES;
-  const int x = blockIdx.y * kTmaCols;
-  const int col = x + lane * 8;
-  const bool active = col < D;
-  // this warp's tokens: n = gw + t * GW for t = 0 .. cnt-1
-  const int64_t GW = static_cast<int64_t>(gridDim.x) * kTmaWarps;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kTmaWarps + warp;
-  const int64_t cnt = gw < N ? (N - 1 - gw) / GW + 1 : 0;
-  // ids of tokens [32b, 32b + 32): lane j holds token 32b + j's ids (idA: current block, idB: next)
-  int idA[LC], idB[LC];
-  auto load_block = [&](int64_t b, int (&dst)[LC]) {
-    const int64_t t = b * 32 + lane;
-    const int64_t n = gw + t * GW;
-#pragma unroll
-    for (int l = 0; l < LC; ++l) dst[l] = t < cnt ? __ldg(ids + n * LC + l) : 0;
-  };
-  load_block(0, idA);
-  load_block(1, idB);
-  bool bad = false;
-  // token t's ids, from the lane that holds them (block cur_block in idA, the next one in idB)
-  auto fetch_ids = [&](int64_t t, int64_t cur_block, int (&out)[LC]) {
-    const int src = static_cast<int>(t & 31);
-    const bool next = (t >> 5) != cur_block;
-#pragma unroll
-    for (int l = 0; l < LC; ++l) {
-      const int a = __shfl_sync(0xffffffffu, idA[l], src);
-      const int b = __shfl_sync(0xffffffffu, idB[l], src);
-      out[l] = next ? b : a;
-    }
-  };
-  // lane 0 issues token t into stage t % DEPTH
-  auto issue_token = [&](int64_t t, const int (&tid)[LC]) {
-    const int s = static_cast<int>(t % C::DEPTH);
-    uint8_t *dst = ring + s * C::STAGE;
-    int32_t row[C::G4 * 4];
-#pragma unroll
-    for (int l = 0; l < C::G4 * 4; ++l) {
-      const bool real = l < LC;
-      const int id = real ? tid[l] : 0;
-      const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(K);
-      bad |= real && !ok;
-      row[l] = (real ? l : 0) * K + (ok ? id : 0);
-    }
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&full[warp][s], C::STAGE);
-#pragma unroll
-    for (int q = 0; q < C::G4; ++q)
-      tma_gather4(&tm, &full[warp][s], dst + q * 4 * kTmaCols * 2, x, row[4 * q], row[4 * q + 1], row[4 * q + 2],
-                  row[4 * q + 3]);
-  };
-  // prologue: the first DEPTH tokens (all in block 0: DEPTH < 32)
-  static_assert(C::DEPTH < 32, "the prologue takes its ids from the first block of 32 tokens");
-  int64_t issued = 0;
-  for (int64_t t = 0; t < C::DEPTH && t < cnt; ++t) {
-    int tid[LC];
-    fetch_ids(t, 0, tid);
-    if (lane == 0) issue_token(t, tid);
-    ++issued;
-  }
-  bool ok = true;
-  for (int64_t t = 0; t < cnt; ++t) {
-    const int64_t blk = t >> 5;
-    const int s = static_cast<int>(t % C::DEPTH);
-    const uint32_t parity = static_cast<uint32_t>((t / C::DEPTH) & 1);
-    int tid[LC];
-    fetch_ids(t, blk, tid);  // this token's ids (validity of each row)
-    if (!mbar_wait(&full[warp][s], parity, &abort_flag)) {
-      ok = false;
-      break;
-    }
-    float acc[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-    const uint8_t *st = ring + s * C::STAGE + lane * 16;
-#pragma unroll
-    for (int l = 0; l < LC; ++l) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(st + l * kTmaCols * 2);
-      if (static_cast<unsigned>(tid[l]) < static_cast<unsigned>(K)) {
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
-          acc[2 * k] += f.x;
-          acc[2 * k + 1] += f.y;
-        }
-      }
-    }
-    if (active) {
-      float4 *dst = reinterpret_cast<float4 *>(recon + (gw + t * GW) * D + col);
-      __stcs(dst, make_float4(acc[0], acc[1], acc[2], acc[3]));
-      __stcs(dst + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
-    }
-    fence_proxy_async_smem();  // this lane's reads of stage s are ordered before its refill
-    __syncwarp();
-    const int64_t tn = t + C::DEPTH;
-    if (tn < cnt) {
-      int nid[LC];
-      fetch_ids(tn, blk, nid);
-      if (lane == 0) issue_token(tn, nid);
-      ++issued;
-    }
-    if ((t & 31) == 31) {  // the next block becomes current; load the one after it
-#pragma unroll
-      for (int l = 0; l < LC; ++l) idA[l] = idB[l];
-      load_block(blk + 2, idB);
-    }
-  }
-  if (!ok) {
-    abort_flag = 1;
-    set_status(status, RVQ_ERR_TIMEOUT);
-    // no bulk copy may still be in flight when the block exits: wait (bounded) for the issued ones
-    if (lane == 0) {
-      int never = 0;
-      for (int64_t t = issued - C::DEPTH < 0 ? 0 : issued - C::DEPTH; t < issued; ++t)
-        mbar_wait(&full[warp][static_cast<int>(t % C::DEPTH)], static_cast<uint32_t>((t / C::DEPTH) & 1), &never);
-    }
-  }
-  if (bad && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
-}
-
-typedef CUresult (*DecodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline DecodeTiledFn decode_tiled_fn() {
-  static DecodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<DecodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// RVQ_DECODE_TMA=1 selects the TMA gather kernel for bf16 codebooks (tuning knob; off by default:
-// on 2^20 tokens x 8 levels of [8,16384,1024] bf16 codebooks it took 3.13 ms against 1.76 ms for
-// the register-gather kernel).
-inline bool tma_decode_enabled() {
-  static int v = [] {
-    const char *e = getenv("RVQ_DECODE_TMA");
-    return e ? atoi(e) : 0;
-  }();
-  return v != 0;
-}
-
-template <int LC>
-cudaError_t launch_tma_t(const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon, int32_t *status,
-                         cudaStream_t s) {
-  using C = TmaCfg<LC>;
-  DecodeTiledFn fn = decode_tiled_fn();
-  if (!fn) return cudaErrorUnknown;
-  static int attr_ok = -1;
-  if (attr_ok < 0)
-    attr_ok = cudaFuncSetAttribute(decode_tma_kernel<LC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) ==
-              cudaSuccess;
-  if (attr_ok != 1) return cudaErrorUnknown;
-  CUtensorMap tm;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(LC) * K};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {kTmaCols, 1};
-  cuuint32_t estr[2] = {1, 1};
-  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(cb), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorUnknown;
-  int sms = 0;
-  if (device_sm_count(&sms) != RVQ_OK) return cudaErrorUnknown;
-  const int64_t gx = std::min<int64_t>((N + kTmaWarps - 1) / kTmaWarps, sms);
-  const int gy = D / kTmaCols;
-  if (gy > 65535) return cudaErrorInvalidValue;
-  return launch_pdl(decode_tma_kernel<LC>, dim3(static_cast<unsigned>(gx), gy), dim3(kTmaWarps * 32),
-                    static_cast<size_t>(C::SMEM), s, tm, ids, N, K, D, recon, status);
-}
-
-template <int LC = 1>
-cudaError_t dispatch_tma(int L, const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon,
-                         int32_t *status, cudaStream_t s) {
-  if constexpr (LC > 16) {
-    return cudaErrorInvalidValue;
-  } else {
-    if (L == LC) return launch_tma_t<LC>(ids, N, cb, K, D, recon, status, s);
-    return dispatch_tma<LC + 1>(L, ids, N, cb, K, D, recon, status, s);
-  }
-}
-
 template <bool CB_BF16, int VEC, int LC>
 cudaError_t launch_fixed(const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon, int32_t *status,
                          cudaStream_t s) {
@@ -484,14 +245,6 @@ int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_d
   if (N == 0) return RVQ_OK;
   if (L <= 16) {
     cudaError_t e;
-    // the TMA gather needs whole 256-column slices, a row coordinate range within int32, and rows
-    // addressable as a 2-D tensor (16-byte aligned base, checked by the caller)
-    if (cb_dtype == RVQ_BF16 && D % kTmaCols == 0 && static_cast<int64_t>(L) * K < (int64_t(1) << 31) &&
-        tma_decode_enabled()) {
-      e = dispatch_tma(L, ids, N, cb, K, D, recon, status, s);
-      note_launch();
-      return e == cudaSuccess ? RVQ_OK : e == cudaErrorInvalidValue ? RVQ_ERR_UNSUPPORTED : RVQ_ERR_CUDA;
-    }
     if (cb_dtype == RVQ_BF16)
       e = (D % 8 == 0 && kBf16Vec == 8) ? dispatch_fixed<true, 8>(L, ids, N, cb, K, D, recon, status, s)
                                         : dispatch_fixed<true, 4>(L, ids, N, cb, K, D, recon, status, s);

@@ -6,34 +6,43 @@
 // level): for every level l, every row takes the codeword nearest (squared Euclidean, lowest
 // index on ties) to its running residual and subtracts it.
 //
-// Per level the engine runs three kernels on the caller's stream:
+// Engine.  Both paths score with the same distance GEMM tile: s = r~ . c~ for a 128-row x 256-codeword
+// tile as a dense bf16 GEMM with fp32 accumulation, operands moved by TMA (cp.async.bulk.tensor,
+// 128B swizzle) into a shared-memory ring, tcgen05.mma issued by one thread into a double-buffered
+// TMEM accumulator (2 x 256 columns).  One extra K=16 step adds ||c||^2/2 (split into three bf16
+// parts) and the main steps negate A, so TMEM holds d~/2 = ||c||^2/2 - r~.c~ directly.  Epilogue
+// warps read it with tcgen05.ld (one TMEM lane = one row) and keep a running top-8 (d~, id) per
+// row; the distance matrix never leaves the SM.
 //
-//  1. dist_topk_kernel (tensor cores).  Scores s = r~ . c~ for all (row, codeword) pairs as a
-//     dense bf16 GEMM [N,D] x [D,K] -> fp32, tile 128 rows x 256 codewords, operands moved by
-//     TMA into a 4-stage shared-memory ring (128B swizzle), tcgen05.mma issued by one thread
-//     into a double-buffered TMEM accumulator (2 x 256 columns).  Four epilogue warps read the
-//     accumulator with tcgen05.ld (one TMEM lane = one row per thread), form the approximate
-//     shifted distance d~ = ||c||^2 - 2 s and keep a sorted running top-8 per row.  The distance
-//     matrix never leaves the SM.  A persistent grid of G CTAs splits the (row tile, codeword
-//     tile) units into G contiguous ranges, so the grid is balanced for any N; a CTA writes one
-//     partial top-8 list per row tile it touched.
-//  2. rescore_kernel (one warp per row).  Merges the partial lists, bounds the bf16 error E of
-//     every d~ from per-row and per-level norms, rescans exactly (fp64 accumulation of fp32
-//     differences) every candidate within 2E of the best, and accepts the exact minimum when
-//     it is provably below every non-candidate (certificate: best - ||r||^2 < T - E, T = the
-//     smallest d~ that was not kept).  Accepted rows write their id and update r -= C_l[id]
-//     (fp32) and the bf16 operand copy for the next level.  Other rows are queued.
-//  3. fallback_kernel.  Queued rows get an exact scan of all K codewords (fp64 accumulation)
-//     and the same update.
+//  * encode_flow_kernel (D in (128, 256] or (512, 1024]): every level in ONE cooperative launch,
+//    one CTA per SM.  The level loop is a dataflow over 128-row tiles: GEMM chunks of (level l,
+//    row tile rt) start as soon as the certificate warps have settled level l-1 of rt (counter
+//    cert_done[l-1][rt]); the certificate warps take (l, rt) once all its chunks are written
+//    (chunk_done[l][rt]).  Per CTA: a TMA producer warp, an MMA-issuer warp, a norm-split warp,
+//    8 epilogue warps and 4 (D = 1024) or 3 (D = 256) certificate warps.  Rows the certificate
+//    cannot settle get an exact scan of all K codewords, cut into slices any certificate warp may
+//    run.  Every wait is bounded (status RVQ_ERR_TIMEOUT when nothing moved for two seconds).
+//  * other widths (and RVQ_PERSISTENT=0): per level, dist_topk_kernel (persistent GEMM + top-8 over
+//    contiguous ranges of (row tile, codeword tile) units, 4 or 8 epilogue warps), then
+//    rescore_fast_kernel / rescore_kernel (certificate, one warp per row) and
+//    fallback_fast_kernel / fallback_kernel (exact scan of the rows the certificate left).
 //
-// Error bound used by the certificate, per row and level (r fp32 residual, r~ = bf16(r),
-// c stored codeword, c~ = bf16(c), n = fl32(||c||^2), s~ = tensor-core r~.c~ with fp32
-// accumulation, gamma = (D+16) 2^-22):
+// Certificate (rescore_row): the candidate lists of a row are merged, every approximate distance
+// carries the bf16 error bound E below, every candidate within 2E of the best is rescored exactly
+// (fp32 differences, fp64 sums), and the exact minimum (ties: lowest id) is accepted when
+// best - ||r||^2 < T - E, T being the smallest approximate distance some list dropped.  Accepted
+// rows update r -= C_l[id] in fp32 and write the next level's bf16 operand and row statistics.
+//
+// Error bound, per row and level (r fp32 residual, r~ = bf16(r), c stored codeword, c~ = bf16(c),
+// n = fl32(||c||^2), gamma = (D+32) 2^-22; Cmax, dCmax, C~max, Nmax the per-level maxima of ||c||,
+// ||c-c~||, ||c~||, n from rvq_build_norms):
 //   | (||r-c||^2 - ||r||^2) - d~ | <= (D/32+2) 2^-24 Nmax + 2 (||r-r~|| Cmax + ||r~|| dCmax)
-//                                     + 2 gamma ||r~|| C~max + 2^-23 (Nmax + 2 ||r~|| C~max)
-// where Cmax, dCmax, C~max, Nmax are the per-level maxima of ||c||, ||c-c~||, ||c~||, n from
-// rvq_build_norms (Cauchy-Schwarz on the two rounding error vectors, worst-case summation error
-// of the fp32 accumulator, rounding of n and of the epilogue FMA), inflated by 1%.
+//                                     + 2 gamma (||r~|| C~max + 0.51 Nmax) + 2^-23 Nmax
+// (Cauchy-Schwarz on the two rounding-error vectors, a worst-case bound of fp32 accumulation of
+// D products and three norm parts with truncation allowed, the fp32 norm sums and the three-part
+// bf16 split of n/2), inflated by 1%.  It assumes that the tensor core forms bf16 products
+// exactly and adds them into the fp32 accumulator with at most one rounding (or truncation) per
+// addition; a GPU test measures |d~ - exact| against E on the workloads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -72,17 +81,12 @@ constexpr uint16_t BF16_BIG = 0x7F7F;  // largest finite bf16: codeword columns 
 
 __device__ __forceinline__ float inf_f() { return __int_as_float(0x7f800000); }
 constexpr float kPastK = 3.0e38f;  // key of a column past K (never a real half-distance)
-#ifndef RVQ_MERGE_LANES
-#define RVQ_MERGE_LANES 10
-#endif
-constexpr int kMergeLanes = RVQ_MERGE_LANES;  // lanes needing inserts that switch a chunk to merging
+constexpr int kMergeLanes = 10;  // lanes needing inserts that switch a chunk to merging
 __device__ __forceinline__ double inf_d() { return __longlong_as_double(0x7ff0000000000000LL); }
 
 // Thread organisation of the distance-GEMM block: EPI epilogue warps (EPI/4 column groups x 4
 // TMEM lane quadrants), then the TMA producer warp, the MMA-issuer warp and the norm-split warp.
-// PAIR: the block is one CTA of a 2-CTA cluster that shares a 256-row x 256-codeword tile
-// (tcgen05 cta_group::2, M=256): each CTA loads its own 128 rows and 128 of the 256 codewords.
-template <int EPI, bool PAIR>
+template <int EPI>
 struct GemmCfg {
   static constexpr int GROUPS = EPI / 4;
   static constexpr int COLS = BN / GROUPS;  // columns of a tile one epilogue thread scans
@@ -92,9 +96,8 @@ struct GemmCfg {
   static constexpr int PRODUCER = EPI;
   static constexpr int ISSUER = EPI + 1;
   static constexpr int SPLITTER = EPI + 2;
-  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // codeword rows this CTA loads per tile
-  static constexpr int STAGE = A_BYTES + B_ROWS * BK * 2;
-  static constexpr int NSTAGE = PAIR ? (EPI >= 16 ? 5 : 6) : (EPI >= 16 ? 3 : 4);
+  static constexpr int STAGE = A_BYTES + BN * BK * 2;
+  static constexpr int NSTAGE = EPI >= 16 ? 3 : 4;
   static constexpr int AUG_A_OFF = NSTAGE * STAGE;
   static constexpr int AUG_B_OFF = AUG_A_OFF + AUG_A_BYTES;                // 2 slots
   static constexpr int MERGE_OFF = AUG_B_OFF + 2 * AUG_B_BYTES;            // (GROUPS-1) x 128 x 8 x 8 B
@@ -116,8 +119,8 @@ struct GemmArgs {
   int32_t *status;
   int32_t *zero_counter;  // set to 0 by the first thread (the level's fallback counter), or null
 };
-// Units are (row tile, codeword tile) pairs; a row tile is 128 rows, or 256 for CTA pairs, and the
-// U units are split into G contiguous ranges, one per CTA (or per CTA pair).
+// Units are (row tile, codeword tile) pairs of 128 rows x 256 codewords; the U units are split into
+// G contiguous ranges, one per CTA.
 
 // CTA that owns unit u when U units are split into G contiguous ranges [cU/G, (c+1)U/G).
 __host__ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t U, int G) {
@@ -250,11 +253,11 @@ __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
 }
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
-template <int EPI, bool PAIR>
-__global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
+template <int EPI>
+__global__ void __launch_bounds__(GemmCfg<EPI>::THREADS, 1)
     dist_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs a) {
-  using C = GemmCfg<EPI, PAIR>;
+  using C = GemmCfg<EPI>;
   constexpr int NSTAGE = C::NSTAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -275,12 +278,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = the pair's leader (issues the MMAs)
-  const int64_t cid = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  const int64_t cid = blockIdx.x;
   const int64_t u0 = cid * a.U / a.G;
   const int64_t u1 = (cid + 1) * a.U / a.G;
   const int KB = a.D / BK;
-  constexpr int UNIT_ROWS = PAIR ? 2 * BM : BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -289,8 +290,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], (PAIR ? 2 : 1) * C::EPI_THREADS);
-      mbar_init(&afull[b], PAIR ? 64 : 32);
+      mbar_init(&tempty[b], C::EPI_THREADS);
+      mbar_init(&afull[b], 32);
     }
     mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
     mbar_init(mdone, 128);
@@ -308,25 +309,13 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
   }
   fence_proxy_async_smem();
   if (warp == C::ISSUER) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(tmem_holder, TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_holder, TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
-  if constexpr (PAIR)
-    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  // the leader's barriers as seen from either CTA of the pair
-  const uint32_t full_l = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
-  const uint32_t tempty_l = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
-  const uint32_t afull_l = PAIR ? mapa_shared(smem_u32(afull), 0) : 0u;
   griddep_launch_dependents();
   griddep_wait();  // the residual operand and candidate buffers belong to the previous kernel until here
   if (a.zero_counter && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_counter = 0;
@@ -343,23 +332,17 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
       for (int64_t u = u0; u < u1 && ok; ++u) {
         const int64_t rt = u / a.Tc;
         const int ct = static_cast<int>(u - rt * a.Tc);
-        const int32_t row0 = static_cast<int32_t>(rt * UNIT_ROWS + rank * BM);
-        const int32_t cw0 = ct * BN + static_cast<int32_t>(rank) * C::B_ROWS;
+        const int32_t row0 = static_cast<int32_t>(rt * BM);
+        const int32_t cw0 = ct * BN;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t *sa = smem + s * C::STAGE;
-          if constexpr (PAIR) {  // both CTAs' bytes complete the leader's barrier
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
-            tma_load_2d_pair(&tmA, full_l + s * 8, sa, kb * BK, row0);
-            tma_load_2d_pair(&tmB, full_l + s * 8, sa + A_BYTES, kb * BK, cw0);
-          } else {
-            mbar_arrive_expect_tx(&full[s], C::STAGE);
-            tma_load_2d(&tmA, &full[s], sa, kb * BK, row0);
-            tma_load_2d(&tmB, &full[s], sa + A_BYTES, kb * BK, cw0);
-          }
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          tma_load_2d(&tmA, &full[s], sa, kb * BK, row0);
+          tma_load_2d(&tmB, &full[s], sa + A_BYTES, kb * BK, cw0);
           ++issued;
           if (++s == NSTAGE) {
             s = 0;
@@ -370,9 +353,8 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
       if (!ok) {
         *abort_flag = 1;
         set_status(a.status, RVQ_ERR_TIMEOUT);
-        // no bulk copy may still be landing in shared memory when the block exits (a pair's
-        // bytes are counted on the leader's barriers, so the leader drains for both)
-        const int64_t pending = (PAIR && rank != 0) ? 0 : (issued < NSTAGE ? issued : NSTAGE);
+        // no bulk copy may still be landing in shared memory when the block exits
+        const int64_t pending = issued < NSTAGE ? issued : NSTAGE;
         for (int64_t j = 0; j < pending; ++j) {
           int back = s - 1 - static_cast<int>(j);
           uint32_t p = ph;
@@ -391,9 +373,9 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
     for (int64_t u = u0; u < u1; ++u, ++i) {
       const int slot = static_cast<int>(i & 1);
       const int ct = static_cast<int>(u - (u / a.Tc) * a.Tc);
-      constexpr int GROUPS_B = C::B_ROWS / 8;                       // row groups this CTA holds
+      constexpr int GROUPS_B = BN / 8;  // row groups of the tile
       const bool writer = lane < GROUPS_B;
-      const int c0 = ct * BN + static_cast<int>(rank) * C::B_ROWS + lane * 8;  // row group `lane`
+      const int c0 = ct * BN + lane * 8;  // row group `lane`
       float h[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) h[j] = (writer && c0 + j < a.K) ? 0.5f * __ldg(a.norms + c0 + j) : 0.f;
@@ -421,20 +403,17 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
         dst[j] = make_uint4(h1 | (static_cast<uint32_t>(h2) << 16), h3, 0, 0);
       }
       fence_proxy_async_smem();
-      if constexpr (PAIR)
-        mbar_arrive_cluster(afull_l + slot * 8);
-      else
-        mbar_arrive(&afull[slot]);
+      mbar_arrive(&afull[slot]);
     }
     if (!ok) {
       *abort_flag = 1;
       set_status(a.status, RVQ_ERR_TIMEOUT);
     }
   } else if (warp == C::ISSUER) {
-    // ------------------------------------------------------------ MMA issuer (the pair's leader)
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc_main = idesc_bf16_f32(UNIT_ROWS, BN, true);  // accumulates -r~.c~
-      constexpr uint32_t idesc_aug = idesc_bf16_f32(UNIT_ROWS, BN, false);  // + ||c||^2 / 2
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main = idesc_bf16_f32(BM, BN, true);  // accumulates -r~.c~
+      constexpr uint32_t idesc_aug = idesc_bf16_f32(BM, BN, false);  // + ||c||^2 / 2
       const uint64_t adesc_aug = sdesc_k_noswizzle(smem_u32(aug_a), 128, 256);
       int s = 0;
       uint32_t ph = 0;
@@ -450,10 +429,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
         tc_fence_after();
         const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
         const uint64_t bdesc_aug = sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128);
-        if constexpr (PAIR)
-          umma_f16_pair(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
-        else
-          umma_f16(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
+        umma_f16(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
@@ -466,34 +442,22 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k) {
             const uint64_t step = static_cast<uint64_t>(k * UK * 2 / 16);
-            if constexpr (PAIR)
-              umma_f16_pair(dt, ad + step, bd + step, idesc_main, 1u);
-            else
-              umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
+            umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
           }
-          if constexpr (PAIR)
-            umma_commit_pair_mc(&empty[s], 0x3);  // frees the stage in both CTAs
-          else
-            umma_commit(&empty[s]);
+          umma_commit(&empty[s]);
           if (++s == NSTAGE) {
             s = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        if constexpr (PAIR)
-          umma_commit_pair_mc(&tfull[buf], 0x3);  // both CTAs' epilogues may read their TMEM
-        else
-          umma_commit(&tfull[buf]);
+        umma_commit(&tfull[buf]);
       }
       if (!ok) {
         *abort_flag = 1;
         set_status(a.status, RVQ_ERR_TIMEOUT);
       }
-      if constexpr (PAIR)
-        umma_commit_pair(mma_done);
-      else
-        umma_commit(mma_done);
+      umma_commit(mma_done);
       mbar_wait(mma_done, 0, never);
     }
   } else {
@@ -537,11 +501,10 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
       }
       ++nflush;
       if (grp == 0) {
-        const int64_t rt128 = rt * (UNIT_ROWS / BM) + rank;  // this CTA's 128-row tile
-        const int64_t n = rt128 * BM + row_in_tile;
+        const int64_t n = rt * BM + row_in_tile;
         if (n < a.N) {
           const int slot = static_cast<int>(cid) - cta_of_unit(rt * a.Tc, a.U, a.G);
-          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt128 * a.maxs + slot) * BM + row_in_tile) * TOPK);
+          float4 *out = reinterpret_cast<float4 *>(a.cand + ((rt * a.maxs + slot) * BM + row_in_tile) * TOPK);
 #pragma unroll
           for (int t = 0; t < TOPK; ++t)
             if (bi[t] >= a.K) {  // a past-K key kept only because the range had < 8 codewords
@@ -591,10 +554,7 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
         tmem_ld_wait();
         if (ch == C::CHUNKS - 1) {
           tc_fence_before();
-          if constexpr (PAIR)
-            mbar_arrive_cluster(tempty_l + buf * 8);
-          else
-            mbar_arrive(&tempty[buf]);
+          mbar_arrive(&tempty[buf]);
         }
         const int c0 = col0 + ct0;
         float d[32];
@@ -630,17 +590,11 @@ __global__ void __launch_bounds__(GemmCfg<EPI, PAIR>::THREADS, 1)
 
   tc_fence_before();
   __syncwarp();
-  if constexpr (PAIR)
-    cluster_sync();  // neither CTA leaves while the leader's MMAs may still use its memory
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   if (warp == C::ISSUER) {
     __syncwarp();
-    if constexpr (PAIR)
-      tmem_dealloc_pair(tmem_base, TMEM_COLS);
-    else
-      tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -741,7 +695,6 @@ struct RowArgs {
   int64_t N;
   int D, K, L, l;
   int Tc, G, maxs;
-  int pair;  // units span 256 rows (CTA pairs) instead of 128
   int64_t U;
   int64_t rt0;  // first row tile of the unit range, else 0
   int nslots;   // > 0: every row tile has exactly nslots candidate lists (all-levels kernel)
@@ -838,7 +791,7 @@ __global__ void __launch_bounds__(256) rescore_kernel(const RowArgs a) {
   if (n >= a.N) return;
   const int64_t rt = n / BM;
   const int rin = static_cast<int>(n - rt * BM);
-  const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;  // the unit row tile this 128-row tile belongs to
+  const int64_t ut = rt - a.rt0;  // the unit row tile this 128-row tile belongs to
   const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
   const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
   const int ncand = (c1 - c0 + 1) * TOPK;
@@ -1028,7 +981,7 @@ __device__ __forceinline__ bool rescore_row(const RowArgs &a, int64_t n, int lan
   const int rin = static_cast<int>(n - rt * BM);
   int ncand = a.nslots * TOPK;
   if (a.nslots <= 0) {
-    const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;
+    const int64_t ut = rt - a.rt0;
     const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
     const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
     ncand = (c1 - c0 + 1) * TOPK;
@@ -1450,7 +1403,7 @@ __device__ __forceinline__ void exact_slice(const RowArgs &a, int64_t n, int k0,
 // the MMA issuer or, when set, the TMA producer.
 template <int EPI, int RW, int SKIP>
 struct FlowCfg {
-  static constexpr int THREADS = GemmCfg<EPI, false>::THREADS + RW * 32;
+  static constexpr int THREADS = GemmCfg<EPI>::THREADS + RW * 32;
   static constexpr int CERT0 = EPI + 3;  // first of the RW warps after the GEMM roles
   static constexpr int CERT_WARPS = RW - __builtin_popcount(SKIP);
 };
@@ -1460,7 +1413,7 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     encode_flow_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB3, const GemmArgs a, const RowArgs r0,
                        const FlowArgs fa) {
-  using C = GemmCfg<EPI, false>;
+  using C = GemmCfg<EPI>;
   constexpr int NSTAGE = C::NSTAGE;
   constexpr int CERT0 = FlowCfg<EPI, RW, SKIP>::CERT0;
   constexpr int CW = FlowCfg<EPI, RW, SKIP>::CERT_WARPS;
@@ -2036,9 +1989,8 @@ struct Plan {
   int64_t RT;  // 128-row tiles
   int Tc;
   int64_t U;
-  int G;       // CTAs, or CTA pairs when pair
+  int G;       // CTAs
   int maxs;    // partial-list slots per row tile (the larger of the two paths' needs)
-  bool pair;
   // all levels in one cooperative launch (encode_flow_kernel)
   bool flow;
   int L;
@@ -2057,16 +2009,6 @@ inline bool persistent_enabled() {
   return v != 0;
 }
 
-// RVQ_FLOW_NC=n (1..16) fixes the chunks per row tile of the all-levels kernel (tuning knob).
-inline int flow_chunks_forced() {
-  static int v = [] {
-    const char *e = getenv("RVQ_FLOW_NC");
-    const int n = e ? atoi(e) : 0;
-    return n >= 1 && n <= MAX_SLOTS ? n : 0;
-  }();
-  return v;
-}
-
 // Row chunks (float4 per lane) of the register-resident row kernels for feature width D <= 1024.
 inline int row_chunks(int D) { return D <= 128 ? 1 : D <= 256 ? 2 : D <= 512 ? 4 : 8; }
 
@@ -2077,33 +2019,11 @@ inline int64_t slots_needed(int64_t U, int64_t G, int64_t Tc) {
   return std::min<int64_t>(G, 1 + (Tc - 1 + f - 1) / f);
 }
 
-// CTA pairs (tcgen05 cta_group::2) halve the codeword traffic per SM.  Off unless RVQ_PAIR=1
-// (tuning knob): on the measured workloads the single-CTA kernel is not L2-bound.
-inline bool use_pairs(int64_t N) {
-  static int forced = [] {
-    const char *e = getenv("RVQ_PAIR");
-    return e ? (atoi(e) != 0 ? 1 : 0) : -1;
-  }();
-  return forced >= 0 ? forced == 1 : false;  // measured: no gain over single CTAs at D = 256, 1024
-}
-
-int resident_pair_clusters(int D);
-
 inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
-  const int sms0 = sms;
   Plan p;
-  p.pair = use_pairs(N);
-  if (p.pair) {
-    const int clusters = resident_pair_clusters(D);
-    if (clusters < 1)
-      p.pair = false;
-    else
-      sms = std::min(sms / 2, clusters);
-  }
   p.RT = (N + BM - 1) / BM;
   p.Tc = (K + BN - 1) / BN;
-  const int64_t unit_rows = p.pair ? 2 * BM : BM;
-  p.U = ((N + unit_rows - 1) / unit_rows) * p.Tc;
+  p.U = p.RT * p.Tc;
   // every CTA covers at least f = floor(U/G) units, so a row tile (Tc consecutive units) meets
   // at most 1 + ceil((Tc-1)/f) CTAs; keep that within the rescore warp's candidate capacity
   const int64_t slots_cap = MAX_SLOTS;
@@ -2117,14 +2037,13 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
   p.L = L;
   // D in (128, 256] and (512, 1024]: 8 epilogue + 5 certificate warps (other widths run the
   // levels one by one)
-  p.flow = !p.pair && D <= 1024 && (nch == 2 || nch == 8) && persistent_enabled() &&
+  p.flow = D <= 1024 && (nch == 2 || nch == 8) && persistent_enabled() &&
            static_cast<uint64_t>(N) * static_cast<uint64_t>(L) < (uint64_t(1) << 32);
   p.NC = p.S = p.RPT = p.NS = p.slice = p.Gf = 0;
   if (p.flow) {
-    p.Gf = sms0;
+    p.Gf = sms;
     // enough chunks per level to keep every CTA busy and finish a row tile soon after it starts
     int nc = static_cast<int>(std::min<int64_t>(MAX_SLOTS, std::max<int64_t>(1, (4 * p.Gf + p.RT - 1) / p.RT)));
-    if (flow_chunks_forced() > 0) nc = flow_chunks_forced();
     nc = std::min(nc, p.Tc);
     p.S = (p.Tc + nc - 1) / nc;
     p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
@@ -2224,85 +2143,42 @@ inline bool make_map(CUtensorMap *m, const void *base, int64_t rows, int D, int 
 }
 
 
-template <int EPI, bool PAIR>
+template <int EPI>
 inline bool set_gemm_attr() {
-  return cudaFuncSetAttribute(dist_topk_kernel<EPI, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<EPI, PAIR>::SMEM) == cudaSuccess;
+  return cudaFuncSetAttribute(dist_topk_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<EPI>::SMEM) == cudaSuccess;
 }
 
 // Epilogue warps of the per-level distance GEMM: 4 above D = 512 (a tile's longer MMA hides a
 // 4-warp epilogue: 5% faster than 8 at D = 1024), else 8 (8 beat 16 at D = 256: 31.4 vs 35.0 ms
-// per offline level, and 4: 33.2 ms).  RVQ_EPI_WARPS=4|8|16 overrides the choice (tuning knob).
-inline int epilogue_warps(int D) {
-  static int forced = [] {
-    const char *e = getenv("RVQ_EPI_WARPS");
-    const int v = e ? atoi(e) : 0;
-    return (v == 4 || v == 8 || v == 16) ? v : 0;
-  }();
-  if (forced) return forced;
-  return D > 512 ? 4 : 8;
-}
+// per offline level, and 4: 33.2 ms).
+inline int epilogue_warps(int D) { return D > 512 ? 4 : 8; }
 
 inline bool gemm_attrs_ready(int epi) {
   static std::once_flag once;
   static bool ok = false;
   std::call_once(once, [] {
-    ok = set_gemm_attr<4, false>() && set_gemm_attr<8, false>() && set_gemm_attr<16, false>() &&
-         set_gemm_attr<4, true>() && set_gemm_attr<8, true>() && set_gemm_attr<16, true>();
+    ok = set_gemm_attr<4>() && set_gemm_attr<8>();
   });
   (void)epi;
   return ok;
 }
 
-template <int EPI, bool PAIR>
+template <int EPI>
 inline cudaError_t launch_gemm_t(int groups, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
                                  const GemmArgs &ga) {
-  using C = GemmCfg<EPI, PAIR>;
+  using C = GemmCfg<EPI>;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(groups * (PAIR ? 2 : 1));
+  cfg.gridDim = dim3(groups);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = PAIR ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, dist_topk_kernel<EPI, PAIR>, tmA, tmB, ga);
-}
-
-// Clusters of two GEMM CTAs that can be resident at once (an SM pair must share a GPC).
-template <int EPI>
-inline int max_pair_clusters() {
-  static int n = [] {
-    using C = GemmCfg<EPI, true>;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2);
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, dist_topk_kernel<EPI, true>, &cfg) != cudaSuccess) clusters = 0;
-    return clusters;
-  }();
-  return n;
-}
-
-// Resident CTA-pair clusters for the epilogue width that feature width D selects.
-inline int resident_pair_clusters(int D) {
-  if (!gemm_attrs_ready(0)) return 0;
-  const int epi = epilogue_warps(D);
-  return epi == 4 ? max_pair_clusters<4>() : epi == 16 ? max_pair_clusters<16>() : max_pair_clusters<8>();
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dist_topk_kernel<EPI>, tmA, tmB, ga);
 }
 
 // All-levels dataflow encode, instantiated for 2 (D in (128, 256]) and 8 (D in (512, 1024])
@@ -2311,7 +2187,7 @@ inline int resident_pair_clusters(int D) {
 template <int EPI, int RW, int SK, bool CB, bool XB, int NCH>
 inline bool set_flow_attr() {
   return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, SK, CB, XB, NCH>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<EPI, false>::SMEM) == cudaSuccess;
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<EPI>::SMEM) == cudaSuccess;
 }
 
 inline bool flow_attrs_ready() {
@@ -2334,7 +2210,7 @@ inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tm
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(FlowCfg<EPI, RW, SK>::THREADS);
-  cfg.dynamicSmemBytes = GemmCfg<EPI, false>::SMEM;
+  cfg.dynamicSmemBytes = GemmCfg<EPI>::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: CTAs wait on one another's counters
@@ -2362,16 +2238,10 @@ inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cud
                 : launch_flow_t<EW, RWD, SW, false, false, 8>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
 }
 
-inline cudaError_t launch_gemm(int epi, bool pair, int groups, cudaStream_t s, const CUtensorMap &tmA,
-                               const CUtensorMap &tmB, const GemmArgs &ga) {
-  if (pair) {
-    if (epi == 4) return launch_gemm_t<4, true>(groups, s, tmA, tmB, ga);
-    if (epi == 16) return launch_gemm_t<16, true>(groups, s, tmA, tmB, ga);
-    return launch_gemm_t<8, true>(groups, s, tmA, tmB, ga);
-  }
-  if (epi == 4) return launch_gemm_t<4, false>(groups, s, tmA, tmB, ga);
-  if (epi == 16) return launch_gemm_t<16, false>(groups, s, tmA, tmB, ga);
-  return launch_gemm_t<8, false>(groups, s, tmA, tmB, ga);
+inline cudaError_t launch_gemm(int epi, int groups, cudaStream_t s, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                               const GemmArgs &ga) {
+  if (epi == 4) return launch_gemm_t<4>(groups, s, tmA, tmB, ga);
+  return launch_gemm_t<8>(groups, s, tmA, tmB, ga);
 }
 
 }  // namespace enc
@@ -2398,6 +2268,19 @@ extern "C" int rvq_encode_levels_per_launch(int64_t N, int D, int L, int K, int 
   if (st != RVQ_OK) return st;
   const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, L, sms);
   *levels = p.flow ? L : 1;
+  return RVQ_OK;
+}
+
+extern "C" int rvq_encode_candidate_layout(int64_t N, int D, int L, int K, size_t *offset, int *slots) {
+  using namespace rvq;
+  if (!offset || !slots || N < 0 || D < 1 || L < 1 || K < 1) return RVQ_ERR_ARG;
+  if (L > 64 || D < 64 || D > 4096 || D % 64 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  int sms = 0;
+  int st = device_sm_count(&sms);
+  if (st != RVQ_OK) return st;
+  const enc::Plan p = enc::make_plan(std::max<int64_t>(N, 1), K, D, L, sms);
+  *offset = enc::make_layout(N, D, p).cand;
+  *slots = p.maxs;
   return RVQ_OK;
 }
 
@@ -2497,7 +2380,6 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     r0.Tc = p.Tc;
     r0.G = p.Gf;
     r0.maxs = p.maxs;
-    r0.pair = 0;
     r0.U = 0;
     r0.rt0 = 0;
     r0.nslots = p.NC;
@@ -2546,7 +2428,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   for (int l = 0; l < L && !all_levels; ++l) {
     const size_t lvl = static_cast<size_t>(l) * K * D * 2;
     CUtensorMap tmB;
-    if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, p.pair ? BN / 2 : BN)) return RVQ_ERR_CUDA;
+    if (!make_map(&tmB, static_cast<const uint8_t *>(op) + lvl, K, D, BN)) return RVQ_ERR_CUDA;
     GemmArgs ga;
     ga.norms = norms + static_cast<size_t>(l) * K;
     ga.N = N;
@@ -2560,7 +2442,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ga.status = status;
     ga.zero_counter = (fast && l == 0) ? fb_count : nullptr;
     profile_begin(s);
-    const cudaError_t ge = launch_gemm(epi, p.pair, p.G, s, (x_is_operand && l == 0) ? tmX : tmA, tmB, ga);
+    const cudaError_t ge = launch_gemm(epi, p.G, s, (x_is_operand && l == 0) ? tmX : tmA, tmB, ga);
     profile_end(s);
     note_launch();
     if (ge != cudaSuccess) return RVQ_ERR_CUDA;
@@ -2574,7 +2456,6 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     ra.Tc = p.Tc;
     ra.G = p.G;
     ra.maxs = p.maxs;
-    ra.pair = p.pair ? 1 : 0;
     ra.U = p.U;
     ra.rt0 = 0;
     ra.nslots = 0;
@@ -2634,18 +2515,50 @@ namespace enc {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[RVQ_NOALLOC_SCRATCH_BYTES];
 
 // Device address of the scratch array on the current device (host code cannot use the symbol
-// itself), looked up once per device with that device current.
+// itself).  It is looked up with that device current the first time the device is used, and again
+// whenever the device's current context is a different one (cudaDeviceReset destroys the primary
+// context, and the module, with the array in it, is loaded anew at another address).  Contexts are
+// told apart by their process-unique id (cuCtxGetId), so a handle value reused by a later context
+// cannot bring back a stale address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+inline bool current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 inline int noalloc_scratch(void **ptr) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void *addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RVQ_ERR_CUDA;
   std::lock_guard<std::mutex> g(mu);
-  if (!addr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);  // false before the runtime made a context current
+  if (!addr[dev] || !have_ctx || ctx != ctx_of[dev]) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RVQ_ERR_CUDA;
+    if (!current_context_id(&ctx)) return RVQ_ERR_CUDA;  // the lookup made the primary context current
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *ptr = addr[dev];
   return RVQ_OK;
@@ -2729,7 +2642,7 @@ template <bool CB_BF16, int SRC, int NCH>
 __device__ __forceinline__ void shard_best_row(const RowArgs &a, int64_t k0, double2 *sel, int64_t n, int lane) {
   const int64_t rt = n / BM;
   const int rin = static_cast<int>(n - rt * BM);
-  const int64_t ut = (a.pair ? (rt >> 1) : rt) - a.rt0;
+  const int64_t ut = rt - a.rt0;
   const int c0 = cta_of_unit(ut * a.Tc, a.U, a.G);
   const int c1 = cta_of_unit(ut * a.Tc + a.Tc - 1, a.U, a.G);
   const int ncand = (c1 - c0 + 1) * TOPK;
@@ -3026,7 +2939,7 @@ extern "C" int rvq_shard_select(const void *features, int f_dtype, int64_t N, in
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, x_is_operand ? features : static_cast<const void *>(Rt), N, D, BM)) return RVQ_ERR_CUDA;
   if (!make_map(&tmB, static_cast<const uint8_t *>(op) + static_cast<size_t>(l) * K_shard * D * 2, K_shard, D,
-                p.pair ? BN / 2 : BN))
+                BN))
     return RVQ_ERR_CUDA;
   const int epi = epilogue_warps(D);
   if (!gemm_attrs_ready(epi)) return RVQ_ERR_CUDA;
@@ -3043,7 +2956,7 @@ extern "C" int rvq_shard_select(const void *features, int f_dtype, int64_t N, in
   ga.status = status;
   ga.zero_counter = fb_count;  // this call's count of exact shard scans
   profile_begin(s);
-  const cudaError_t ge = launch_gemm(epi, p.pair, p.G, s, tmA, tmB, ga);
+  const cudaError_t ge = launch_gemm(epi, p.G, s, tmA, tmB, ga);
   profile_end(s);
   note_launch();
   if (ge != cudaSuccess) return RVQ_ERR_CUDA;
@@ -3057,7 +2970,6 @@ extern "C" int rvq_shard_select(const void *features, int f_dtype, int64_t N, in
   ra.Tc = p.Tc;
   ra.G = p.G;
   ra.maxs = p.maxs;
-  ra.pair = p.pair ? 1 : 0;
   ra.U = p.U;
   ra.rt0 = 0;
   ra.nslots = 0;

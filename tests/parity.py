@@ -8,7 +8,10 @@ legitimate near-tie can send two encoders down different residual paths):
     oracle's best-vs-second gap is below REL_GAP relative, and there the GPU's chosen
     distance must be within REL_GAP relative of the minimum (an exact 0 minimum needs 0).
   * the free-running oracle ids are also compared; rows that differ must have taken an
-    exemption at the first level where they differ.
+    exemption at the first level where they differ.  A row whose every level matched the
+    teacher-forced argmin is on the free-running path by construction (same residual, same
+    argmin, level by level, in the same fp64 arithmetic), so only rows with an exemption are
+    re-encoded free-running.
 Reconstructions: ||recon_gpu - recon_oracle(ids_gpu)|| <= REL_L2 * ||recon_oracle|| per row,
 and the residual within REL_L2 * ||x|| of x - recon_oracle(ids_gpu).  fp32 accumulation of
 L <= 16 codewords carries a relative error of a few 1e-7, so 1e-5 has ample headroom.
@@ -43,8 +46,11 @@ def check_ids(x, C, rows, ids_gpu, threads=0):
             f"row {rows[j]} level {l}: gpu id {g[j, l]} (d={chosen[j, l]!r}) but oracle argmin "
             f"{tf['argmin'][j, l]} (d={best[j, l]!r}, second={second[j, l]!r}); "
             f"{int(bad.sum())} violations in {bad.size} row-levels")
-    free, _, _, _ = oracle.encode(x, C, rows=rows, threads=threads)
-    differ = (free != g)
+    differ = np.zeros_like(g, dtype=bool)
+    touched = np.where(exempt.any(axis=1))[0]
+    if touched.size:
+        free, _, _, _ = oracle.encode(x, C, rows=rows[touched], threads=threads)
+        differ[touched] = free != g[touched]
     first_diff_ok = True
     for j in np.where(differ.any(axis=1))[0]:
         l = int(np.argmax(differ[j]))

@@ -142,11 +142,9 @@ def test_host_argument_checks(lib):
     assert ebs(16, 5, 2, 8, 16, 16, 16, 256, 100, None, None) == -3                         # too small
 
 
-def test_missing_library_fails_loudly(tmp_path):
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU fallback: without librvq.so the binding raises instead of running anything else."""
+    monkeypatch.setattr(mvt, "_lib", None)
+    monkeypatch.setattr(mvt, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError):
-        mvt._lib_backup = mvt._lib
-        try:
-            mvt._lib = None
-            mvt.load(str(tmp_path / "nope.so"))
-        finally:
-            mvt._lib = mvt._lib_backup
+        mvt.load()
