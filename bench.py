@@ -10,7 +10,11 @@ Metric: tokens (feature vectors) per second, in millions.  `value` is measured w
 inputs resident in HBM; `e2e` repeats it through the same calls with the features copied
 from pinned host memory every step and the ids + decoded recon copied back.
 
-    python bench.py [--gpus N --steps K --warmup W] [--workload image] [--impl reference]
+    python bench.py [--gpus N --steps K --warmup W] [--workload detok] [--impl reference]
+The default workload is the largest single-GPU configuration, `detok`: 2^20 tokens x 8 levels of
+16384 codewords at D = 1024 (bf16 codebooks), decoded to fp32 features that the step re-encodes
+and decodes again.  The encode-only figures of `offline` and `packed` are added to the same line
+(--also).
 Multi-GPU: launched by torchrun, one rank per GPU; every rank quantizes its own batch
 (weak scaling, no data-path collective); times are the max over ranks.
 """
@@ -31,6 +35,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 import workloads  # noqa: E402
+from multimodal_visual_tokenization_b200 import sharding  # noqa: E402
 
 METRIC = "RVQ encode Mtokens/s (L levels, K codes, dim D) and % tensor-core peak; decode GB/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -45,7 +50,9 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    p.add_argument("--workload", default="image", choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--workload", default="detok", choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--also", default="offline,packed",
+                   help="comma-separated workloads whose encode alone is timed in the same run ('none': skip)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -126,6 +133,56 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ replica timing
+
+class EventTimer:
+    """Per-step CUDA events recorded on the launching stream."""
+
+    def __init__(self, steps, stream):
+        import torch
+        self.stream = stream
+        self.starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        self.ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+
+    def start(self, k):
+        self.starts[k].record(self.stream)
+
+    def stop(self, k):
+        self.ends[k].record(self.stream)
+
+    def total_ms(self):
+        self.ends[-1].synchronize()
+        return sum(s.elapsed_time(e) for s, e in zip(self.starts, self.ends))
+
+
+def replica_measure(step, steps, timer, units, between=None, sync=None, device=None):
+    """Time `steps` steps of this rank's replica: a barrier and a sync on both sides, `between`
+    (the L2 flush) outside each step's timer.  Returns (ms_per_step, value, total_ms): the total
+    is the max over ranks, value = the units all ranks processed per step / ms_per_step (units/s)."""
+    import torch.distributed as dist
+    grouped = dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1
+    if sync:
+        sync()
+    if grouped:
+        dist.barrier()
+    if sync:
+        sync()
+    for k in range(steps):
+        if between:
+            between()
+        timer.start(k)
+        step()
+        timer.stop(k)
+    if sync:
+        sync()
+    if grouped:
+        dist.barrier()
+    total_ms = sharding.max_over_ranks(timer.total_ms(), device)
+    all_units = sharding.sum_over_ranks(float(units), device)
+    ms_per_step = total_ms / steps
+    return ms_per_step, all_units / (ms_per_step / 1e3), total_ms
+
+
 # ------------------------------------------------------------------ helpers
 
 def gpu_index(local_rank):
@@ -154,37 +211,53 @@ def read_traffic(workload, kernel):
     return None
 
 
-def cpu_baseline(g, seconds, rows_hint=None):
-    """The fp64 oracle, as it stands, on a bounded seeded row sample on this host's cores."""
+def cpu_model():
+    """The host CPU's model string (logged beside the oracle's figures)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_rows(g, rows):
+    """Feature rows of the workload as the oracle gets them (detok: decoded from the planted ids)."""
     import oracle
-    x, C = g["x"], g["codebooks"]
+    if g["x"] is not None:
+        return np.ascontiguousarray(g["x"][rows])
+    return oracle.decode(g["planted"][rows], g["codebooks"]).astype(np.float32)
+
+
+def cpu_baseline(g, seconds, threads=0):
+    """The fp64 oracle, as it stands, on a bounded seeded row sample on this host's cores: per row the
+    step's work, the greedy encode of all L levels and the decode of the ids it chose.  Rows are
+    independent, so the sample's tokens/s is the whole batch's.  threads=0: all cores (OpenMP
+    default); the thread setting is restored afterwards."""
+    import oracle
+    C = g["codebooks"]
     spec = g["spec"]
-    if x is None:  # detok: the CPU leg decodes
-        ids = g["planted"]
-        probe = workloads.sample_rows(len(ids), 256, seed=9)
-        t0 = time.perf_counter()
-        oracle.decode(ids[probe], C)
-        dt = max(time.perf_counter() - t0, 1e-6)
-        rows = min(len(ids), max(256, int(len(probe) * seconds / dt)))
-        sample = workloads.sample_rows(len(ids), rows, seed=10)
-        t0 = time.perf_counter()
-        oracle.decode(ids[sample], C)
-        dt = time.perf_counter() - t0
-    else:
-        cores = oracle.threads()
-        probe = workloads.sample_rows(len(x), cores, seed=8)
-        t0 = time.perf_counter()
-        oracle.encode(x, C, rows=probe)
-        dt = max(time.perf_counter() - t0, 1e-6)
-        rows = int(max(cores, min(len(x), len(probe) * seconds / dt)))
-        rows = max(1, min(len(x), rows if rows_hint is None else rows_hint))
-        sample = workloads.sample_rows(len(x), rows, seed=10)
-        t0 = time.perf_counter()
-        oracle.encode(x, C, rows=sample)
-        dt = time.perf_counter() - t0
-    value = len(sample) / dt / 1e6
-    return {"value": value, "unit": "Mtokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{len(sample)} of {spec.N} rows (seeded), full pipeline per row, "
+    default = oracle.threads(0)
+    cores = oracle.threads(threads) if threads > 0 else default
+    try:
+        def run(rows):
+            xs = oracle_rows(g, rows)          # input preparation, not timed
+            t0 = time.perf_counter()
+            ids, _, _, _ = oracle.encode(xs, C)
+            oracle.decode(ids, C)
+            return time.perf_counter() - t0
+        probe = workloads.sample_rows(spec.N, cores, seed=8)
+        dt = max(run(probe), 1e-6)
+        rows = int(max(cores, min(spec.N, len(probe) * seconds / dt)))
+        sample = workloads.sample_rows(spec.N, rows, seed=10)
+        dt = run(sample)
+    finally:
+        oracle.threads(default)
+    return {"value": len(sample) / dt / 1e6, "unit": "Mtokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} of {spec.N} rows (seeded), encode of all levels + decode per row, "
                       f"fp64 plain C + OpenMP over rows, {dt:.2f} s"}
 
 
@@ -203,6 +276,8 @@ def run_reference(args, rank, world):
         cb = cpu_baseline(g, per_step)
         if k >= args.warmup:
             vals.append(cb["value"])
+    cb["cpu_model"] = cpu_model()
+    cb["host_cpus"] = os.cpu_count()
     value = statistics.median(vals)
     line = {"metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": spec.N / (value * 1e6) * 1e3, "higher_is_better": True,
@@ -217,11 +292,54 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ our arm
 
+def encode_figures(name, dev, peaks, flush_l2, reps=3):
+    """rvq_encode alone on another workload (inputs resident, L2 flushed before each timed call):
+    time, tokens/s and the distance GEMM's share of the bf16 peaks."""
+    import torch
+
+    import multimodal_visual_tokenization_b200 as mvt
+    g = workloads.generate(name)
+    spec = g["spec"]
+    N, D, L, K = spec.N, spec.D, spec.L, spec.K
+    cb = torch.from_numpy(g["codebooks"]).to(dev)
+    if spec.cb_dtype == "bf16":
+        cb = cb.to(torch.bfloat16)
+    x = torch.from_numpy(g["x"]).to(dev)
+    if spec.f_dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    tok = mvt.Tokenizer(cb)
+    off = torch.from_numpy(g["offsets"]).to(dev)
+    fb = torch.zeros(L, dtype=torch.int32, device=dev)
+    out = {"ids": torch.empty((N, L), dtype=torch.int32, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(2):
+        tok.encode(x, offsets=off, out=out, fallbacks=fb)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        fb.zero_()
+        flush_l2()
+        e0.record(stream)
+        tok.encode(x, offsets=off, out=out, fallbacks=fb, check=False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.median(ts)
+    tflops = 2.0 * N * K * D * L / (ms / 1e3) / 1e12
+    sus = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    code, lpl = mvt.rvq_encode_levels_per_launch(N, D, L, K)
+    return {"workload": workload_label(spec), "N": N, "D": D, "L": L, "K": K, "encode_ms": ms,
+            "Mtok_per_s": N / (ms / 1e3) / 1e6, "tflops": tflops, "frac_sustained": tflops / sus,
+            "frac_burst": tflops / burst, "fallbacks_per_level": fb.cpu().tolist(),
+            "kernel": "encode_flow_kernel" if lpl > 1 else "dist_topk_kernel per level",
+            "timing": f"median of {reps} calls, L2 flushed before each"}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
     import multimodal_visual_tokenization_b200 as mvt
-    from multimodal_visual_tokenization_b200 import sharding
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -281,21 +399,13 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
 
     # -------------------------------------------------- timed region, device-resident inputs
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
+    timer = EventTimer(args.steps, stream)
     with ClockSampler(gpu_index(local_rank)) as clk:
         in_timed = args.gemm_events == "timed"
         mvt.rvq_profile_enable(in_timed)
         launches0 = mvt.rvq_launch_count()
-        for k in range(args.steps):
-            flush_l2()
-            starts[k].record(stream)
-            step(x)
-            ends[k].record(stream)
-        torch.cuda.synchronize(dev)
+        ms_per_step, value, total_ms = replica_measure(lambda: step(x), args.steps, timer, N, between=flush_l2,
+                                                       sync=lambda: torch.cuda.synchronize(dev), device=dev)
         launches = mvt.rvq_launch_count() - launches0
         if not in_timed:  # the same steps again, GEMM launches bracketed by events
             mvt.rvq_profile_enable(True)
@@ -305,15 +415,10 @@ def run_ours(args, rank, world, local_rank):
             torch.cuda.synchronize(dev)
         code, gemm_n, gemm_ms = mvt.rvq_profile_read()
         mvt.rvq_profile_enable(False)
-    if world > 1:
-        torch.distributed.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sharding.max_over_ranks(sum(step_ms), dev)
     st = int(status.item())
     if st != 0:
         raise mvt.RVQError(st, "device status during the timed region")
-    ms_per_step = total_ms / args.steps
-    value = N * world / (ms_per_step / 1e3) / 1e6
+    value /= 1e6  # tokens/s -> Mtokens/s
 
     # -------------------------------------------------- per-call breakdown (separate pass)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -335,7 +440,8 @@ def run_ours(args, rank, world, local_rank):
     breakdown = {k: statistics.median(v) for k, v in br.items()}
     s_cb = 2 if spec.cb_dtype == "bf16" else 4
     # algorithmic minimum of a decode: ids read once, every referenced codeword row read once, recon
-    # written once (a small batch references only part of the codebooks)
+    # written once.  When every codeword is referenced (detok) this is N*L*4 + L*K*D*s + N*D*4; a
+    # small batch (image) references only part of the codebooks.
     ids_h = ids.cpu().numpy()
     rows_used = sum(int(np.unique(ids_h[:, l]).size) for l in range(L))
     decode_bytes = N * L * 4 + rows_used * D * s_cb + N * D * 4
@@ -548,9 +654,12 @@ def run_ours(args, rank, world, local_rank):
                "pipeline": "2 buffer sets; copy-in, compute and copy-out streams overlap across steps"}
 
     # -------------------------------------------------- roofline of the distance GEMM
+    # a step longer than 20 ms runs under the power cap: the sustained bf16 figure is its peak; the
+    # fraction of the burst figure is reported beside it
     long_step = ms_per_step > 20.0
     peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
     peak = float(peaks.get(peak_key, PEAKS_FALLBACK[peak_key]))
+    peak_burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
     # the dominant encode kernel: one launch per level (distance GEMM + top-8), or one launch for
     # all levels (dataflow kernel: GEMM, top-8, certificate and residual update)
     code, lpl = mvt.rvq_encode_levels_per_launch(N, D, L, K)
@@ -563,6 +672,7 @@ def run_ours(args, rank, world, local_rank):
     traffic = read_traffic(args.workload, kernel)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
+                "frac_burst": achieved / peak_burst, "peak_burst": peak_burst,
                 "kernel": kernel, "levels_per_launch": lpl, "launch_ms": launch_ms,
                 "launches_timed": enc_launches, "flops_per_launch": flops_per_launch,
                 "peak_source": f"{peak_src} {peak_key}"}
@@ -573,14 +683,19 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         rows = workloads.sample_rows(N, 6, seed=11)
-        xs = g["x"] if not detok_only else x.cpu().numpy()
-        want, _, _, _ = oracle.encode(xs, g["codebooks"], rows=rows)
+        xs = x[torch.from_numpy(rows).to(dev)].float().cpu().numpy()   # the rows the GPU encoded
+        want, _, _, _ = oracle.encode(xs, g["codebooks"])
         got = ids.cpu().numpy()[rows]
         parity = {"rows": int(len(rows)), "ids_equal_oracle": bool(np.array_equal(want, got))}
-        gg = dict(g)
-        if detok_only:
-            gg["x"] = xs
-        cpu = cpu_baseline(gg, args.cpu_seconds)
+        cpu = cpu_baseline(g, args.cpu_seconds)
+        one = cpu_baseline(g, min(args.cpu_seconds, 8.0), threads=1)
+        cpu.update({"value_1thread": one["value"], "sample_1thread": one["sample"], "cpu_model": cpu_model(),
+                    "host_cpus": os.cpu_count()})
+
+    also = {}
+    if world == 1 and args.also != "none" and args.rows is None:
+        for name in [w for w in args.also.split(",") if w and w != args.workload]:
+            also[name] = encode_figures(name, dev, peaks, flush_l2)
 
     clocks = clk.summary()
     line = {
@@ -604,6 +719,7 @@ def run_ours(args, rank, world, local_rank):
         **({"pack": pack} if pack is not None else {}),
         **({"sharded": sharded} if sharded is not None else {}),
         **({"codebook_update": kmeans} if kmeans is not None else {}),
+        **({"encode_other_workloads": also} if also else {}),
         "fallbacks_per_level": fb.cpu().tolist(),
         "parity_sample": parity,
     }
