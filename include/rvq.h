@@ -32,6 +32,11 @@
  *     Read it after synchronising the stream.
  *   - Inputs must be finite.  Calls that overlap on the GPU must not share output or
  *     workspace buffers.
+ *   - Every compute entry point opens an NVTX range named after itself (visible to nsys / ncu).
+ *   - Host-side fault injection, for testing a caller's error handling without a GPU fault:
+ *     with RVQ_FAULT="<entry point>:<status>[,...]" in the environment (read once, at the first
+ *     call), each named entry point returns that negative rvq_status at once, before it checks
+ *     its arguments or touches the device.  E.g. RVQ_FAULT="rvq_encode:-4,rvq_decode:-5".
  */
 #ifndef RVQ_H_
 #define RVQ_H_

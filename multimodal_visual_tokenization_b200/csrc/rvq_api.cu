@@ -1,6 +1,11 @@
-// rvq_api.cu -- status strings, the launch counter and the distance-GEMM profiling hooks.
+// rvq_api.cu -- status strings, the launch counter, the distance-GEMM profiling hooks and the
+// host-side fault injection switch.
 #include <atomic>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
+#include <string>
+#include <utility>
 #include <vector>
 
 #include "rvq.h"
@@ -17,6 +22,30 @@ int device_sm_count(int *sms) {
   if (cudaGetDevice(&dev) != cudaSuccess) return RVQ_ERR_CUDA;
   if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return RVQ_ERR_CUDA;
   return RVQ_OK;
+}
+
+int injected_fault(const char *entry) {
+  static const std::vector<std::pair<std::string, int>> faults = [] {
+    std::vector<std::pair<std::string, int>> v;
+    const char *e = getenv("RVQ_FAULT");
+    std::string spec = e ? e : "";
+    size_t pos = 0;
+    while (pos < spec.size()) {
+      size_t end = spec.find(',', pos);
+      if (end == std::string::npos) end = spec.size();
+      const std::string item = spec.substr(pos, end - pos);
+      const size_t colon = item.rfind(':');
+      if (colon != std::string::npos) {
+        const int code = atoi(item.c_str() + colon + 1);
+        if (code < 0 && code >= RVQ_ERR_TIMEOUT) v.emplace_back(item.substr(0, colon), code);
+      }
+      pos = end + 1;
+    }
+    return v;
+  }();
+  for (const auto &f : faults)
+    if (f.first == entry) return f.second;
+  return 0;
 }
 
 namespace {

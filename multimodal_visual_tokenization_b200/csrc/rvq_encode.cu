@@ -2248,6 +2248,7 @@ inline cudaError_t launch_gemm(int epi, int groups, cudaStream_t s, const CUtens
 }  // namespace rvq
 
 extern "C" int rvq_encode_workspace_size(int64_t N, int D, int L, int K, size_t *bytes) {
+  RVQ_ENTRY("rvq_encode_workspace_size");
   using namespace rvq;
   if (!bytes || N < 0 || D < 1 || L < 1 || K < 1) return RVQ_ERR_ARG;
   if (L > 64 || D < 64 || D > 4096 || D % 64 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
@@ -2289,6 +2290,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
                           const int64_t *offsets, int64_t B, int32_t *ids, float *residual, float *recon,
                           int32_t *fallbacks, void *workspace, size_t workspace_bytes, int32_t *status,
                           void *stream) {
+  RVQ_ENTRY("rvq_encode");
   using namespace rvq;
   using namespace rvq::enc;
   if (N < 0 || D < 1 || L < 1 || K < 1 || B < 0) return RVQ_ERR_ARG;
@@ -2571,6 +2573,7 @@ extern "C" int rvq_encode_noalloc(const void *features, int f_dtype, int64_t N, 
                                   int cb_dtype, const void *cb_operand, const float *norms, const float *level_stats,
                                   int L, int K, const int64_t *offsets, int64_t B, int32_t *ids, float *residual,
                                   float *recon, int32_t *fallbacks, int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_encode_noalloc");
   size_t need = 0;
   int st = rvq_encode_workspace_size(N, D, L, K, &need);
   if (st != RVQ_OK) return st;
@@ -2878,6 +2881,7 @@ inline bool shard_width_ok(int D) { return D >= 64 && D <= 1024 && D % 64 == 0; 
 }  // namespace rvq
 
 extern "C" int rvq_shard_workspace_size(int64_t N, int D, int K_shard, size_t *bytes) {
+  RVQ_ENTRY("rvq_shard_workspace_size");
   using namespace rvq;
   if (!bytes || N < 0 || D < 1 || K_shard < 1) return RVQ_ERR_ARG;
   if (!enc::shard_width_ok(D) || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
@@ -2894,6 +2898,7 @@ extern "C" int rvq_shard_select(const void *features, int f_dtype, int64_t N, in
                                 const float *shard_stats, int L, int K_shard, int64_t k0, int l, float *residual,
                                 double *sel, int32_t *fallbacks, void *workspace, size_t workspace_bytes,
                                 int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_shard_select");
   using namespace rvq;
   using namespace rvq::enc;
   if (N < 0 || D < 1 || L < 1 || K_shard < 1 || k0 < 0 || l < 0 || l >= L) return RVQ_ERR_ARG;
@@ -3013,6 +3018,7 @@ extern "C" int rvq_shard_apply(const void *features, int f_dtype, int64_t N, int
                                const void *const *shard_codebooks, int cb_dtype, const int *shard_K, int L, int l,
                                int32_t *ids, float *residual, void *workspace, size_t workspace_bytes,
                                int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_shard_apply");
   using namespace rvq;
   using namespace rvq::enc;
   if (N < 0 || D < 1 || L < 1 || l < 0 || l >= L || W < 1) return RVQ_ERR_ARG;

@@ -1,9 +1,10 @@
 // rvq_host.h -- host-side helpers shared by the translation units of librvq.so:
-// argument checks, CUDA error mapping, the kernel launch counter and the GEMM
-// profiling events.
+// argument checks, CUDA error mapping, the kernel launch counter, the GEMM
+// profiling events, NVTX ranges and host-side fault injection.
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "rvq.h"
@@ -27,6 +28,25 @@ inline int check_launch() {
 }
 
 int device_sm_count(int *sms);
+
+// NVTX range over one entry-point call, named after the entry point (shown by nsys / ncu
+// timelines; a push and a pop that do nothing while no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
+// Host-side fault injection, for testing how callers handle errors without making a GPU fault:
+// RVQ_FAULT="<entry point>:<status>[,<entry point>:<status>...]" (read once, at the first call)
+// makes each named entry point return that negative rvq_status before it checks its arguments or
+// touches the device.  0 when the entry point is not named (the normal case).
+int injected_fault(const char *entry);
+
+#define RVQ_ENTRY(name)                                        \
+  ::rvq::NvtxRange rvq_nvtx_range_(name);                      \
+  if (const int rvq_fault_ = ::rvq::injected_fault(name)) return rvq_fault_
 
 // Launch with programmatic stream serialization (see griddep_* in rvq_device.cuh).
 template <typename... KArgs, typename... Args>

@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(256) norms_kernel(const void *__restrict__ cb,
 
 extern "C" int rvq_build_norms(const void *codebooks, int cb_dtype, int L, int K, int D, float *norms,
                                float *level_stats, void *cb_operand, void *stream) {
+  RVQ_ENTRY("rvq_build_norms");
   using namespace rvq;
   if (!codebooks || !norms || !level_stats) return RVQ_ERR_ARG;
   if (cb_dtype != RVQ_F32 && cb_dtype != RVQ_BF16) return RVQ_ERR_ARG;

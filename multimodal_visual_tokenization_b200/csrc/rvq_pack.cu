@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(256) gather_sequences_kernel(const int32_t *__
 }  // namespace rvq
 
 extern "C" int rvq_balance_sequences(const int64_t *lengths, int64_t S, int world, int32_t *owner, int64_t *load) {
+  RVQ_ENTRY("rvq_balance_sequences");
   using namespace rvq;
   if (S < 0 || world < 1 || !owner || !load || (S > 0 && !lengths)) return RVQ_ERR_ARG;
   for (int64_t s = 0; s < S; ++s)
@@ -87,6 +88,7 @@ extern "C" int rvq_balance_sequences(const int64_t *lengths, int64_t S, int worl
 extern "C" int rvq_gather_sequences(const int32_t *cache_ids, int L, const int64_t *cache_offsets, int64_t S,
                                     const int64_t *select, int64_t M, const int64_t *out_offsets, int32_t *out_ids,
                                     int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_gather_sequences");
   using namespace rvq;
   if (L < 1 || S < 0 || M < 0) return RVQ_ERR_ARG;
   if (M == 0) return RVQ_OK;

@@ -111,6 +111,7 @@ int launch_scatter(const int32_t *ids, int64_t N, int L, int K, int H, const flo
 
 extern "C" int rvq_embed_backward(const int32_t *ids, int64_t N, int L, int K, int H, const float *grad_out,
                                   float *grad_tables, int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_embed_backward");
   using namespace rvq;
   if (N < 0 || L < 1 || K < 1 || H < 1) return RVQ_ERR_ARG;
   if (L > 64 || H % 4 != 0) return RVQ_ERR_UNSUPPORTED;
@@ -123,6 +124,7 @@ extern "C" int rvq_embed_backward(const int32_t *ids, int64_t N, int L, int K, i
 extern "C" int rvq_codebook_update(const float *points, const int32_t *ids, int64_t N, int D, int K,
                                    const float *old_codebook, float *new_codebook, float *sums, int32_t *counts,
                                    int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_codebook_update");
   using namespace rvq;
   if (N < 0 || D < 1 || K < 1) return RVQ_ERR_ARG;
   if (D % 4 != 0 || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;

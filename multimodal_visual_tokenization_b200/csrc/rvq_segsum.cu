@@ -36,11 +36,12 @@ namespace rvq {
 namespace ss {
 
 constexpr int SS_CH = 8192;    // tokens per histogram / scatter block
-constexpr int SS_COLS = 32;    // gradient columns per slice: 4 lanes x 2 float4 (one 128-byte line of a row)
+constexpr int SS_COLS = 32;    // gradient columns per slice: SS_LPU lanes x 2 float4 of a row
+constexpr int SS_LPU = SS_COLS / 8;  // lanes per run or piece
 constexpr int SS_HOT = 256;    // segments longer than this are summed in pieces of this size
 constexpr int SS_RUN = 256;    // a run of segments is cut where a segment starts in a new window
 constexpr int SS_WARPS = 8;    // warps per block of the sum and fix kernels
-constexpr int SS_UNITS = SS_WARPS * 8;  // runs or pieces per block of the sum kernel (8 per warp)
+constexpr int SS_UNITS = SS_WARPS * 32 / SS_LPU;  // runs or pieces per block of the sum kernel
 constexpr int SS_DEPTH = 8;    // g rows in flight per lane (shared-memory ring of 2 x 16-byte copies)
 constexpr int SS_SUM_SMEM = SS_WARPS * 32 * SS_DEPTH * 32;
 constexpr int SCAN_THREADS = 1024;
@@ -301,9 +302,9 @@ __global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int
   const int64_t s = b / (a.L * per_level);
   const int l = static_cast<int>((b / per_level) % a.L);
   const int64_t ib = b % per_level;
-  const int col = static_cast<int>(s) * SS_COLS + (lane & 3) * 8;  // this lane: col .. col + 7
+  const int col = static_cast<int>(s) * SS_COLS + (lane % SS_LPU) * 8;  // this lane: col .. col + 7
   const bool act0 = col < a.H, act1 = col + 4 < a.H;
-  const int unit = (threadIdx.x >> 2);  // 0 .. SS_UNITS-1
+  const int unit = threadIdx.x / SS_LPU;  // 0 .. SS_UNITS-1
   const int32_t *perm = a.perm + static_cast<int64_t>(l) * a.N;
   const int32_t *nz_start = a.nz_start + static_cast<int64_t>(l) * (a.K + 2);
   const int32_t *m = a.meta + 4 * l;
@@ -480,6 +481,7 @@ bool attrs_ready() {
 }  // namespace rvq
 
 extern "C" int rvq_embed_backward_workspace_size(int64_t N, int L, int K, int H, size_t *bytes) {
+  RVQ_ENTRY("rvq_embed_backward_workspace_size");
   using namespace rvq;
   if (!bytes || N < 0 || L < 1 || K < 1 || H < 1) return RVQ_ERR_ARG;
   if (L > 64 || H % 4 != 0 || K > ss::MAX_K || N >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
@@ -490,6 +492,7 @@ extern "C" int rvq_embed_backward_workspace_size(int64_t N, int L, int K, int H,
 extern "C" int rvq_embed_backward_sorted(const int32_t *ids, int64_t N, int L, int K, int H, const float *grad_out,
                                          float *grad_tables, void *workspace, size_t workspace_bytes,
                                          int32_t *status, void *stream) {
+  RVQ_ENTRY("rvq_embed_backward_sorted");
   using namespace rvq;
   using namespace rvq::ss;
   if (N < 0 || L < 1 || K < 1 || H < 1) return RVQ_ERR_ARG;
