@@ -16,7 +16,7 @@
 //   4. ss_scatter_kernel  per (level, chunk), one warp: tokens in ascending n go to their slots
 //                         (ranks among equal ids from __match_any_sync), so each segment lists its
 //                         tokens in ascending n: a stable counting sort
-//   5. ss_sum_kernel      per (column slice of 32, level): every group of 4 lanes (2 float4 each)
+//   5. ss_sum_kernel      per (column slice of 64, level): every group of 8 lanes (2 float4 each)
 //                         streams the positions of one run in ascending order with SS_DEPTH rows in
 //                         flight per lane (16-byte cp.async copies into a shared-memory ring, so the
 //                         depth costs no registers), and adds each segment's sum into its gradient
@@ -24,9 +24,12 @@
 //                         question arises); a hot id's pieces go to scratch rows instead
 //   6. ss_fix_kernel      per hot id: its pieces summed in order and added into the gradient row
 // Every gradient element is written by one thread, with its terms added in an order fixed by the
-// ids alone, so the result is bit-identical from run to run.  The grid runs slice-major, so the
-// 32-column slice of g being summed for all levels (N x 128 bytes, one line per row) is reused
-// from L2 while it stays there.
+// ids alone, so the result is bit-identical from run to run (and independent of the slice width).
+// The grid runs slice-major, so the slice of g being summed for all levels (N x 256 bytes, two lines
+// per row) is reused from L2 while it stays there.  Slice width, measured on 2^20 Zipf/uniform
+// tokens x 8 levels x 1024 columns: 8 -> 44.3 ms, 16 -> 21.9, 32 -> 10.9, 64 -> 9.0, 128 -> 9.1 (a
+// warp's gathers touch one line per lane group, so narrow slices multiply the lines per gather
+// instruction; wide ones no longer fit L2 between the level passes).
 #include <algorithm>
 
 #include "rvq_device.cuh"
@@ -36,7 +39,7 @@ namespace rvq {
 namespace ss {
 
 constexpr int SS_CH = 8192;    // tokens per histogram / scatter block
-constexpr int SS_COLS = 32;    // gradient columns per slice: SS_LPU lanes x 2 float4 of a row
+constexpr int SS_COLS = 64;    // gradient columns per slice: SS_LPU lanes x 2 float4 of a row
 constexpr int SS_LPU = SS_COLS / 8;  // lanes per run or piece
 constexpr int SS_HOT = 256;    // segments longer than this are summed in pieces of this size
 constexpr int SS_RUN = 256;    // a run of segments is cut where a segment starts in a new window
@@ -291,8 +294,9 @@ __global__ void __launch_bounds__(32) ss_scatter_kernel(const Args a) {
 }
 
 // Block b of the grid: slice s (outermost), level l, then nbu blocks of segments (nz index order)
-// and nbh blocks of hot pieces.  Lane group (lane / 4) owns one segment or piece; its 4 lanes own
-// float4 columns col .. col + 3 of the slice.  Positions are summed one by one in ascending order.
+// and nbh blocks of hot pieces.  Lane group (lane / SS_LPU) owns one run or piece; each of its lanes
+// owns 8 consecutive columns (two float4) of the slice.  Positions are summed one by one in
+// ascending order.
 __global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int nbu, int nbh) {
   griddep_launch_dependents();
   griddep_wait();
