@@ -1251,18 +1251,19 @@ inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blo
 // so level l+1 of a row tile starts while later row tiles of level l are still being scored,
 // and the certificate work runs under the tensor-core work.  Every wait is bounded: it gives up
 // when neither its counter nor the grid's progress word has moved for two seconds.
-// Epilogue and certificate warps of the all-levels kernel.  With the three GEMM-role warps they
-// fill the block to 16 warps (the register budget per thread is set by the warp count rounded up
-// to a multiple of four).  8 + 5 at both widths: at D = 1024, 4 epilogue + 9 certificate warps
-// measured 9% slower on image (the epilogue then shares its SM sub-partition with more
-// certificate work), although 4 epilogue warps are faster in the per-level kernel.
-constexpr int FLOW_EPI_WIDE = 8;
+// Epilogue and certificate warps of the all-levels kernel, after the three GEMM-role warps.
+// D in (512, 1024]: 4 epilogue + 5 more warps (12 per block).  Measured against 8 + 5 (16 warps)
+// with clocks sampled: packed (65503 rows) 1249 vs 1223 TFLOP/s at 1965 MHz, detok (262144 rows)
+// 883 vs 852 TFLOP/s per GHz under the power cap, image unchanged; 4 epilogue + 9 certificate
+// warps in 16 was 9% slower on image.  D in (128, 256]: 8 + 5 (16 warps).
+constexpr int FLOW_EPI_WIDE = 4;
 constexpr int FLOW_RW_WIDE = 5;
 constexpr int FLOW_EPI_NARROW = 8;
 constexpr int FLOW_RW_NARROW = 5;
-// Idle warps among the five (bit i = warp CERT0 + i): at D = 1024 warp 13, which shares the MMA
-// issuer's sub-partition (4 certificate warps; image 13.2 vs 13.1 Mtok/s with 5, 12.8 with 3);
-// at D = 256 also warp 12, the TMA producer's (3 certificate warps; offline 7.61 vs 7.45 with 4).
+// Idle warps among the five (bit i = warp CERT0 + i; warp w runs on SM sub-partition w mod 4): the
+// one that would share the MMA issuer's sub-partition (4 certificate warps; with 8 epilogue warps
+// at D = 1024 image ran 13.2 vs 13.1 Mtok/s with 5, 12.8 with 3); at D = 256 also the TMA
+// producer's (3 certificate warps; offline 7.61 vs 7.45 with 4).
 constexpr int FLOW_SKIP_WIDE = 0b00100;
 constexpr int FLOW_SKIP_NARROW = 0b00110;
 constexpr int EXACT_QCAP = 1024;   // queued rows whose exact scan is split into slices
