@@ -77,6 +77,15 @@ def workload_label(spec):
             f"{spec.f_dtype} features, {spec.cb_dtype} codebooks; {spec.description}")
 
 
+def run_config(spec, world):
+    """The `config` of both arms' lines: the workload and what one step does to it."""
+    return {"workload": workload_label(spec), "N": spec.N, "D": spec.D, "L": spec.L, "K": spec.K,
+            "step": "build codeword norms, encode every row through all L levels (ids + residual), "
+                    "decode the ids",
+            "l2": "flushed between timed steps (GPU arm; the oracle's sample is not L2-resident either)",
+            "parallelism": f"replicas x{world}, rows independent, no data-path collective"}
+
+
 # ------------------------------------------------------------------ clocks during the timed region
 
 class ClockSampler:
@@ -282,9 +291,9 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": spec.N / (value * 1e6) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": workload_label(spec), "N": spec.N, "D": spec.D, "L": spec.L, "K": spec.K,
-                       "note": "fp64 oracle on host cores; each step a bounded seeded row sample; "
-                               "ms_per_step extrapolated to the full batch (rows are independent)"},
+            "config": run_config(spec, world),
+            "note": "fp64 oracle on host cores; each step a bounded seeded row sample; "
+                    "ms_per_step extrapolated to the full batch (rows are independent)",
             "cpu_baseline": dict(cb, value=value),
             "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -569,18 +578,22 @@ def run_ours(args, rank, world, local_rank):
 
         det_ms = time_backward(lambda: check(mvt.rvq_embed_backward_sorted(
             ids_in, N, L, K, D, rec2, gtab, eb_ws, eb_ws_bytes, status, stream), "rvq_embed_backward_sorted"))
-        eb_ms = time_backward(lambda: check(mvt.rvq_embed_backward(ids_in, N, L, K, D, rec2, gtab, status, stream),
+        at_ms = time_backward(lambda: check(mvt.rvq_embed_backward(ids_in, N, L, K, D, rec2, gtab, status, stream),
                                             "rvq_embed_backward"))
         # algorithmic minimum: ids and g read once, every referenced gradient row read and written once
         used = sum(int(np.unique(g["planted"][:, l]).size) for l in range(L))
         eb_bytes = N * L * 4 + N * D * 4 + 2 * used * D * 4
+        # what the sorted kernel has to move: every g row once per level (the rows a level visits are in
+        # id order, so L2 cannot keep them between levels), the gradient rows read and written once
+        moved = N * L * D * 4 + 2 * used * D * 4 + 3 * N * L * 4
         hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-        embed = {"ms": eb_ms, "GB_per_s": eb_bytes / (eb_ms / 1e3) / 1e9, "algorithmic_bytes": eb_bytes,
-                 "frac_hbm": eb_bytes / (eb_ms / 1e3) / 1e9 / hbm,
-                 "fp32x4_atomics_per_s": N * L * (D // 4) / (eb_ms / 1e3),
-                 "kernel": "embed_backward_kernel (fp32x4 atomics)",
-                 "deterministic_ms": det_ms, "deterministic_frac_hbm": eb_bytes / (det_ms / 1e3) / 1e9 / hbm,
-                 "deterministic_kernels": "ss_hist/ss_prefix/ss_scan/ss_scatter (sort by id) + ss_sum + ss_fix",
+        embed = {"ms": det_ms, "GB_per_s": eb_bytes / (det_ms / 1e3) / 1e9, "algorithmic_bytes": eb_bytes,
+                 "frac_hbm": eb_bytes / (det_ms / 1e3) / 1e9 / hbm,
+                 "bytes_moved": moved, "frac_hbm_of_moved": moved / (det_ms / 1e3) / 1e9 / hbm,
+                 "kernels": "ss_hist/ss_prefix/ss_scan/ss_scatter (stable sort by id) + ss_rowsum + ss_fix "
+                            "(deterministic)",
+                 "atomic_ms": at_ms, "atomic_kernel": "embed_backward_kernel (fp32x4 atomics)",
+                 "atomic_frac_hbm": eb_bytes / (at_ms / 1e3) / 1e9 / hbm,
                  "g": "decoded fp32 recon [N,D]"}
         del gtab, eb_ws
 
@@ -702,11 +715,10 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": workload_label(spec), "N": N, "D": D, "L": L, "K": K,
-                   "step": "rvq_build_norms + rvq_encode(ids, residual) + rvq_decode(ids -> recon)",
-                   "gemm_events": args.gemm_events,
-                   "l2": "flushed between timed steps (512 MiB memset + read-back, outside the step events)",
-                   "parallelism": f"replicas x{world}, rows independent, no data-path collective"},
+        "config": run_config(spec, world),
+        "calls": "rvq_build_norms + rvq_encode(ids, residual) + rvq_decode(ids -> recon); L2 flush = 512 MiB "
+                 "memset + read-back outside the step events",
+        "gemm_events": args.gemm_events,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -10,26 +10,24 @@
 //   2. ss_prefix_kernel   per (level, id): the id's count in earlier chunks (so a chunk knows where
 //                         its tokens of that id go) and its total
 //   3. ss_scan_kernel     per level: segment starts (prefix sums of the totals), the list of
-//                         non-empty ids, the "hot" ids (more than SS_HOT tokens) with their pieces
-//                         of SS_HOT positions, and runs: consecutive non-hot segments cut where a
-//                         segment starts in a new window of SS_RUN positions
+//                         non-empty ids and the "hot" ids (more than SS_HOT tokens) with their
+//                         pieces of SS_HOT positions
 //   4. ss_scatter_kernel  per (level, chunk), one warp: tokens in ascending n go to their slots
 //                         (ranks among equal ids from __match_any_sync), so each segment lists its
 //                         tokens in ascending n: a stable counting sort
-//   5. ss_sum_kernel      per (column slice of 64, level): every group of 8 lanes (2 float4 each)
-//                         streams the positions of one run in ascending order with SS_DEPTH rows in
-//                         flight per lane (16-byte cp.async copies into a shared-memory ring, so the
-//                         depth costs no registers), and adds each segment's sum into its gradient
-//                         row with float4 atomics (the only write of those elements, so no ordering
-//                         question arises); a hot id's pieces go to scratch rows instead
+//   5. ss_rowsum_kernel   one warp per (level, segment) or hot piece: the segment's g rows, whole
+//                         (512-byte gathers per instruction), through a per-warp cp.async ring of
+//                         SS_RROWS rows, summed in ascending position order and added into the
+//                         gradient row with float4 atomics (the only write of those elements, so no
+//                         ordering question arises); a hot id's pieces go to scratch rows instead
 //   6. ss_fix_kernel      per hot id: its pieces summed in order and added into the gradient row
 // Every gradient element is written by one thread, with its terms added in an order fixed by the
-// ids alone, so the result is bit-identical from run to run (and independent of the slice width).
-// The grid runs slice-major, so the slice of g being summed for all levels (N x 256 bytes, two lines
-// per row) is reused from L2 while it stays there.  Slice width, measured on 2^20 Zipf/uniform
-// tokens x 8 levels x 1024 columns: 8 -> 44.3 ms, 16 -> 21.9, 32 -> 10.9, 64 -> 9.0, 128 -> 9.1 (a
-// warp's gathers touch one line per lane group, so narrow slices multiply the lines per gather
-// instruction; wide ones no longer fit L2 between the level passes).
+// ids alone, so the result is bit-identical from run to run.  Every g row is read once per level
+// (L x N x H x 4 bytes, from HBM: the rows a level visits are in id order, not in memory order).
+// Measured on 2^20 tokens x 8 levels x 1024 columns (level 0 Zipf(1.1), others uniform): 5.99 ms,
+// against 8.97 ms for a slice-major variant that summed 64-column slices of g (so that a slice could
+// stay in L2 across the level passes; 32-column slices 10.9 ms, 16 -> 21.9, 8 -> 44.3: each gather
+// instruction then touched a line per lane group) and 10.1 ms for the atomic kernel.
 #include <algorithm>
 
 #include "rvq_device.cuh"
@@ -39,14 +37,9 @@ namespace rvq {
 namespace ss {
 
 constexpr int SS_CH = 8192;    // tokens per histogram / scatter block
-constexpr int SS_COLS = 64;    // gradient columns per slice: SS_LPU lanes x 2 float4 of a row
-constexpr int SS_LPU = SS_COLS / 8;  // lanes per run or piece
+constexpr int SS_PAD = 4;      // piece rows (carry) are padded to a multiple of this many columns
 constexpr int SS_HOT = 256;    // segments longer than this are summed in pieces of this size
-constexpr int SS_RUN = 256;    // a run of segments is cut where a segment starts in a new window
-constexpr int SS_WARPS = 8;    // warps per block of the sum and fix kernels
-constexpr int SS_UNITS = SS_WARPS * 32 / SS_LPU;  // runs or pieces per block of the sum kernel
-constexpr int SS_DEPTH = 8;    // g rows in flight per lane (shared-memory ring of 2 x 16-byte copies)
-constexpr int SS_SUM_SMEM = SS_WARPS * 32 * SS_DEPTH * 32;
+constexpr int SS_WARPS = 8;    // warps per block of the fix kernel
 constexpr int SCAN_THREADS = 1024;
 constexpr int MAX_K = 49151;   // K + 1 histogram counters in <= 192 KiB of shared memory
 
@@ -62,16 +55,15 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 struct Layout {
-  int64_t nch, maxp, S, Hpad;
-  size_t hist, start, perm, nz_key, nz_start, run_first, hot_key, hot_p0, meta, carry, total;
+  int64_t nch, maxp, Hpad;
+  size_t hist, start, perm, nz_key, nz_start, hot_key, hot_p0, meta, carry, total;
 };
 
 inline Layout make_layout(int64_t N, int L, int K, int H) {
   Layout w;
   w.nch = (N + SS_CH - 1) / SS_CH;
   w.maxp = std::max<int64_t>(1, 2 * ((N + SS_HOT - 1) / SS_HOT));
-  w.S = (H + SS_COLS - 1) / SS_COLS;
-  w.Hpad = w.S * SS_COLS;
+  w.Hpad = (H + SS_PAD - 1) / SS_PAD * SS_PAD;
   size_t off = 0;
   w.hist = off;      // [L][nch][K+1]: counts, then the id's count in earlier chunks
   off += align256(static_cast<size_t>(L) * w.nch * (K + 1) * 4);
@@ -82,8 +74,6 @@ inline Layout make_layout(int64_t N, int L, int K, int H) {
   w.nz_key = off;    // [L][K+2]: non-empty ids in ascending order (K = out-of-range ids)
   off += align256(static_cast<size_t>(L) * (K + 2) * 4);
   w.nz_start = off;  // [L][K+2]: their segment starts, then N
-  off += align256(static_cast<size_t>(L) * (K + 2) * 4);
-  w.run_first = off; // [L][K+2]: first nz index of every run, then the nz count
   off += align256(static_cast<size_t>(L) * (K + 2) * 4);
   w.hot_key = off;   // [L][K+1]: nz index of every hot segment
   off += align256(static_cast<size_t>(L) * (K + 1) * 4);
@@ -101,8 +91,8 @@ struct Args {
   const int32_t *ids;
   int64_t N;
   int L, K, H;
-  int64_t nch, maxp, S, Hpad;
-  int32_t *hist, *start, *perm, *nz_key, *nz_start, *run_first, *hot_key, *hot_p0, *meta;
+  int64_t nch, maxp, Hpad;
+  int32_t *hist, *start, *perm, *nz_key, *nz_start, *hot_key, *hot_p0, *meta;
   float *carry;
   const float *g;
   float *grad;
@@ -210,7 +200,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) ss_scan_kernel(const Args a) {
   int32_t *nz_start = a.nz_start + static_cast<int64_t>(l) * (a.K + 2);
   int32_t *hot_key = a.hot_key + static_cast<int64_t>(l) * (a.K + 1);
   int32_t *hot_p0 = a.hot_p0 + static_cast<int64_t>(l) * (a.K + 2);
-  const int64_t zb = z;
   for (int k = k0; k < k1; ++k) {
     const int t = start[k];
     start[k] = static_cast<int32_t>(run);
@@ -234,27 +223,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) ss_scan_kernel(const Args a) {
     m[0] = static_cast<int32_t>(tot_nz);
     m[1] = static_cast<int32_t>(tot_hot);
     m[2] = static_cast<int32_t>(tot_pieces);
-  }
-  __syncthreads();  // nz lists complete (block-wide visibility of the global writes)
-  // Runs: a segment starts a new run when it or its predecessor is a breaker (hot, or the bucket of
-  // out-of-range ids: each breaker is a run of its own, skipped by the sum kernel) or when it starts
-  // in another window of SS_RUN positions than its predecessor.
-  auto breaker = [&](int64_t i) {
-    return nz_key[i] >= a.K || nz_start[i + 1] - nz_start[i] > SS_HOT;
-  };
-  auto run_starts = [&](int64_t i) {
-    return i == 0 || breaker(i) || breaker(i - 1) || nz_start[i] / SS_RUN != nz_start[i - 1] / SS_RUN;
-  };
-  int64_t nr = 0;
-  for (int64_t i = zb; i < z; ++i) nr += run_starts(i);
-  int64_t tot_runs;
-  int64_t rb = block_scan(nr, sh, &tot_runs);
-  int32_t *run_first = a.run_first + static_cast<int64_t>(l) * (a.K + 2);
-  for (int64_t i = zb; i < z; ++i)
-    if (run_starts(i)) run_first[rb++] = static_cast<int32_t>(i);
-  if (threadIdx.x == 0) {
-    run_first[tot_runs] = static_cast<int32_t>(tot_nz);
-    a.meta[4 * l + 3] = static_cast<int32_t>(tot_runs);
   }
 }
 
@@ -293,147 +261,112 @@ __global__ void __launch_bounds__(32) ss_scatter_kernel(const Args a) {
   }
 }
 
-// Block b of the grid: slice s (outermost), level l, then nbu blocks of segments (nz index order)
-// and nbh blocks of hot pieces.  Lane group (lane / SS_LPU) owns one run or piece; each of its lanes
-// owns 8 consecutive columns (two float4) of the slice.  Positions are summed one by one in
-// ascending order.
-__global__ void __launch_bounds__(SS_WARPS * 32) ss_sum_kernel(const Args a, int nbu, int nbh) {
+// The sum: one warp per (level, non-empty segment) or hot piece, over all H columns in passes of
+// SS_RCOLS (lane j holds columns 128 q + 4 j .. + 3 of the pass, q = 0 .. 7), so every gather
+// instruction moves 512 contiguous bytes of one g row.  g rows come in through a per-warp cp.async
+// ring of SS_RROWS rows; each lane reads back only the 16-byte pieces it copied itself.  The terms
+// of every element are added in ascending positions of its segment, starting from zero.
+constexpr int SS_RWARPS = 4;    // warps per block
+constexpr int SS_RROWS = 6;     // g rows in flight per warp
+constexpr int SS_RCOLS = 1024;  // columns per pass: 32 lanes x 8 float4
+constexpr int SS_RSMEM = SS_RWARPS * SS_RROWS * SS_RCOLS * 4;
+
+__global__ void __launch_bounds__(SS_RWARPS * 32) ss_rowsum_kernel(const Args a, int64_t units_per_level,
+                                                                   int64_t seg_units) {
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
-  const int64_t per_level = nbu + nbh;
-  const int64_t b = blockIdx.x;
-  const int64_t s = b / (a.L * per_level);
-  const int l = static_cast<int>((b / per_level) % a.L);
-  const int64_t ib = b % per_level;
-  const int col = static_cast<int>(s) * SS_COLS + (lane % SS_LPU) * 8;  // this lane: col .. col + 7
-  const bool act0 = col < a.H, act1 = col + 4 < a.H;
-  const int unit = threadIdx.x / SS_LPU;  // 0 .. SS_UNITS-1
+  const int64_t wg = static_cast<int64_t>(blockIdx.x) * SS_RWARPS + (threadIdx.x >> 5);
+  const int l = static_cast<int>(wg / units_per_level);
+  const int64_t u = wg % units_per_level;
+  if (l >= a.L) return;  // whole warp
   const int32_t *perm = a.perm + static_cast<int64_t>(l) * a.N;
   const int32_t *nz_start = a.nz_start + static_cast<int64_t>(l) * (a.K + 2);
   const int32_t *m = a.meta + 4 * l;
-  const int32_t *nz_key = a.nz_key + static_cast<int64_t>(l) * (a.K + 2);
-  float *grad_l = a.grad + static_cast<int64_t>(l) * a.K * a.H + col;
-  int64_t j0 = 0, j1 = 0;   // positions of this group's run or piece
-  int64_t e = 0;            // end of the current segment (runs)
-  int i = 0, i1 = 0;        // current nz index, end of the run
-  int key = 0;
-  float *piece = nullptr;   // destination of a hot piece's sum
-  if (ib < nbu) {
-    const int64_t r = ib * SS_UNITS + unit;  // run index
-    if (r < __ldg(m + 3)) {
-      const int32_t *run_first = a.run_first + static_cast<int64_t>(l) * (a.K + 2);
-      i = __ldg(run_first + r);
-      i1 = __ldg(run_first + r + 1);
-      key = __ldg(nz_key + i);
-      j0 = __ldg(nz_start + i);
-      e = __ldg(nz_start + i + 1);
-      if (key < a.K && e - j0 <= SS_HOT) j1 = __ldg(nz_start + i1);  // else a breaker: nothing to do
-    }
+  int64_t j0 = 0, j1 = 0;
+  float *dst = nullptr;
+  bool piece = false;
+  if (u < seg_units) {
+    if (u >= __ldg(m)) return;  // beyond the non-empty segments
+    const int key = __ldg(a.nz_key + static_cast<int64_t>(l) * (a.K + 2) + u);
+    j0 = __ldg(nz_start + u);
+    j1 = __ldg(nz_start + u + 1);
+    if (key >= a.K || j1 - j0 > SS_HOT) return;  // out-of-range ids, or a hot id (summed in pieces)
+    dst = a.grad + (static_cast<int64_t>(l) * a.K + key) * a.H;
   } else {
-    const int64_t pi = (ib - nbu) * SS_UNITS + unit;  // piece index
+    const int64_t pi = u - seg_units;  // piece index
     const int nhot = __ldg(m + 1), npieces = __ldg(m + 2);
-    if (pi < npieces) {
-      const int32_t *hot_p0 = a.hot_p0 + static_cast<int64_t>(l) * (a.K + 2);
-      int lo = 0, hi = nhot;  // last h with hot_p0[h] <= pi
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(hot_p0 + mid) <= pi) lo = mid;
-        else hi = mid;
-      }
-      const int zi = __ldg(a.hot_key + static_cast<int64_t>(l) * (a.K + 1) + lo);
-      const int64_t base = __ldg(nz_start + zi), end = __ldg(nz_start + zi + 1);
-      j0 = base + (pi - __ldg(hot_p0 + lo)) * SS_HOT;
-      j1 = min(end, j0 + SS_HOT);
-      e = j1;  // one segment
-      piece = a.carry + (static_cast<int64_t>(l) * a.maxp + pi) * a.Hpad + col;
+    if (pi >= npieces) return;
+    const int32_t *hot_p0 = a.hot_p0 + static_cast<int64_t>(l) * (a.K + 2);
+    int lo = 0, hi = nhot;  // last h with hot_p0[h] <= pi
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(hot_p0 + mid) <= pi) lo = mid;
+      else hi = mid;
     }
+    const int zi = __ldg(a.hot_key + static_cast<int64_t>(l) * (a.K + 1) + lo);
+    const int64_t base = __ldg(nz_start + zi), end = __ldg(nz_start + zi + 1);
+    j0 = base + (pi - __ldg(hot_p0 + lo)) * SS_HOT;
+    j1 = min(end, j0 + SS_HOT);
+    dst = a.carry + (static_cast<int64_t>(l) * a.maxp + pi) * a.Hpad;
+    piece = true;
   }
-  // the segment after the current one (runs only), loaded ahead of its use
-  int nkey = i + 1 < i1 ? __ldg(nz_key + i + 1) : 0;
-  int64_t ne = i + 1 < i1 ? __ldg(nz_start + i + 2) : 0;
-  // Ring of SS_DEPTH slots per lane: position p's 2 x 16 bytes land in slot p % SS_DEPTH, stored
-  // (slot, half, thread) so the lanes of a warp touch consecutive 16-byte words.  Copies are
-  // committed four positions per group, so SS_DEPTH / 4 groups are in flight.
-  constexpr int PF = SS_DEPTH / 4;
-  constexpr int T = SS_WARPS * 32;
-  extern __shared__ float4 ring_all[];
-  float4 *ring = ring_all + threadIdx.x;  // half h of slot t at ring[(2 t + h) * T]
-  const float *gcol = a.g + col;
-  auto issue4 = [&](int64_t p, const int (&nidx)[4]) {
+  // tokens of the (at most SS_HOT = 256) positions: lane j holds position j0 + 32 w + j in tok[w]
+  static_assert(SS_HOT <= 256, "a segment's tokens must fit the 8 windows of 32");
+  int tok[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int t = static_cast<int>((p + u) & (SS_DEPTH - 1));
-      const float *src = gcol + static_cast<int64_t>(nidx[u]) * a.H;
-      if (nidx[u] >= 0 && act0) cp_async16(ring + (2 * t) * T, src);
-      if (nidx[u] >= 0 && act1) cp_async16(ring + (2 * t + 1) * T, src + 4);
-    }
-    cp_async_commit();
-  };
-  auto perm4 = [&](int64_t p, int (&nidx)[4]) {
+  for (int w = 0; w < 8; ++w) tok[w] = j0 + 32 * w + lane < j1 ? __ldg(perm + j0 + 32 * w + lane) : 0;
+  auto token = [&](int64_t p) -> int {
+    const int d = static_cast<int>(p - j0);
+    int t = tok[0];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) nidx[u] = p + u < j1 ? __ldg(perm + p + u) : -1;
+    for (int w = 1; w < 8; ++w)
+      if ((d >> 5) == w) t = tok[w];
+    return __shfl_sync(0xffffffffu, t, d & 31);
   };
+  extern __shared__ float4 rring[];
+  float4 *ring = rring + static_cast<int64_t>(threadIdx.x >> 5) * SS_RROWS * (SS_RCOLS / 4) + lane;
   auto add4 = [](float4 &x, const float4 &y) {
     x.x += y.x;
     x.y += y.y;
     x.z += y.z;
     x.w += y.w;
   };
-  // token indices of the positions issued in the next PF steps (pn[q] holds positions
-  // j + SS_DEPTH + 4q .. during step q of a round of 4 PF positions)
-  int pn[PF][4];
+  for (int c0 = 0; c0 < a.H; c0 += SS_RCOLS) {
+    auto issue = [&](int64_t p) {
+      const int slot = static_cast<int>((p - j0) % SS_RROWS);
+      const float *src = a.g + static_cast<int64_t>(token(p)) * a.H + c0 + 4 * lane;
 #pragma unroll
-  for (int q = 0; q < PF; ++q) {
-    perm4(j0 + 4 * q, pn[q]);
-    issue4(j0 + 4 * q, pn[q]);
-  }
+      for (int q = 0; q < 8; ++q)
+        if (c0 + 128 * q + 4 * lane < a.H) cp_async16(ring + (slot * 8 + q) * 32, src + 128 * q);
+    };
 #pragma unroll
-  for (int q = 0; q < PF; ++q) perm4(j0 + SS_DEPTH + 4 * q, pn[q]);
-  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-  for (int64_t jr = j0; jr < j1; jr += 4 * PF) {
-#pragma unroll
-    for (int q = 0; q < PF; ++q) {
-      const int64_t j = jr + 4 * q;
-      if (j < j1) {
-        cp_async_wait<PF - 1>();  // positions j .. j + 3 have landed
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (j + u < j1) {
-            if (j + u == e) {  // the previous segment of the run is complete: its only write
-              float *d = grad_l + static_cast<int64_t>(key) * a.H;
-              if (act0) atomicAdd(reinterpret_cast<float4 *>(d), acc0);
-              if (act1) atomicAdd(reinterpret_cast<float4 *>(d + 4), acc1);
-              acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
-              acc1 = acc0;
-              ++i;
-              key = nkey;
-              e = ne;
-              if (i + 1 < i1) {
-                nkey = __ldg(nz_key + i + 1);
-                ne = __ldg(nz_start + i + 2);
-              }
-            }
-            const int t = static_cast<int>((j + u) & (SS_DEPTH - 1));
-            if (act0) add4(acc0, ring[(2 * t) * T]);
-            if (act1) add4(acc1, ring[(2 * t + 1) * T]);
-          }
-        }
-        // the slots just read (their values are already in the sums) take positions j + SS_DEPTH ..
-        issue4(j + SS_DEPTH, pn[q]);
-        perm4(j + 2 * SS_DEPTH, pn[q]);
-      }
+    for (int r = 0; r < SS_RROWS - 1; ++r) {
+      if (j0 + r < j1) issue(j0 + r);
+      cp_async_commit();
     }
-  }
-  cp_async_wait<0>();
-  if (j1 > j0) {
-    if (piece) {  // padding columns of a piece row get zeros
-      reinterpret_cast<float4 *>(piece)[0] = acc0;
-      reinterpret_cast<float4 *>(piece)[1] = acc1;
-    } else {
-      float *d = grad_l + static_cast<int64_t>(key) * a.H;
-      if (act0) atomicAdd(reinterpret_cast<float4 *>(d), acc0);
-      if (act1) atomicAdd(reinterpret_cast<float4 *>(d + 4), acc1);
+    float4 acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t p = j0; p < j1; ++p) {
+      if (p + SS_RROWS - 1 < j1) issue(p + SS_RROWS - 1);
+      cp_async_commit();
+      cp_async_wait<SS_RROWS - 1>();  // position p has landed
+      const int slot = static_cast<int>((p - j0) % SS_RROWS);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (c0 + 128 * q + 4 * lane < a.H) add4(acc[q], ring[(slot * 8 + q) * 32]);
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int col = c0 + 128 * q + 4 * lane;
+      if (col >= a.H) continue;
+      float4 *d = reinterpret_cast<float4 *>(dst + col);
+      if (piece)
+        *d = acc[q];
+      else
+        atomicAdd(d, acc[q]);  // the only write of these elements
     }
   }
 }
@@ -476,7 +409,7 @@ bool attrs_ready() {
     const int bytes = (MAX_K + 1) * 4;
     ok = cudaFuncSetAttribute(ss_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
          cudaFuncSetAttribute(ss_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
-         cudaFuncSetAttribute(ss_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SS_SUM_SMEM) == cudaSuccess;
+         cudaFuncSetAttribute(ss_rowsum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SS_RSMEM) == cudaSuccess;
   }
   return ok == 1;
 }
@@ -517,14 +450,12 @@ extern "C" int rvq_embed_backward_sorted(const int32_t *ids, int64_t N, int L, i
   a.H = H;
   a.nch = w.nch;
   a.maxp = w.maxp;
-  a.S = w.S;
   a.Hpad = w.Hpad;
   a.hist = reinterpret_cast<int32_t *>(ws + w.hist);
   a.start = reinterpret_cast<int32_t *>(ws + w.start);
   a.perm = reinterpret_cast<int32_t *>(ws + w.perm);
   a.nz_key = reinterpret_cast<int32_t *>(ws + w.nz_key);
   a.nz_start = reinterpret_cast<int32_t *>(ws + w.nz_start);
-  a.run_first = reinterpret_cast<int32_t *>(ws + w.run_first);
   a.hot_key = reinterpret_cast<int32_t *>(ws + w.hot_key);
   a.hot_p0 = reinterpret_cast<int32_t *>(ws + w.hot_p0);
   a.meta = reinterpret_cast<int32_t *>(ws + w.meta);
@@ -541,16 +472,15 @@ extern "C" int rvq_embed_backward_sorted(const int32_t *ids, int64_t N, int L, i
       launch_pdl(ss_scan_kernel, dim3(L), dim3(SCAN_THREADS), 0, s, a) != cudaSuccess ||
       launch_pdl(ss_scatter_kernel, chunks, dim3(32), hsm, s, a) != cudaSuccess)
     return RVQ_ERR_CUDA;
-  const int64_t seg_max = std::min<int64_t>(static_cast<int64_t>(K) + 1, N);  // runs <= non-empty ids
-  const int nbu = static_cast<int>((seg_max + SS_UNITS - 1) / SS_UNITS);
-  const int nbh = static_cast<int>((w.maxp + SS_UNITS - 1) / SS_UNITS);
-  const int64_t sum_blocks = w.S * L * static_cast<int64_t>(nbu + nbh);
+  const int64_t seg_max = std::min<int64_t>(static_cast<int64_t>(K) + 1, N);  // non-empty ids (with the bucket)
   const int hot_max = static_cast<int>(std::min<int64_t>(K, N / SS_HOT + 1));
   const int64_t fix_blocks = (static_cast<int64_t>(L) * hot_max + SS_WARPS - 1) / SS_WARPS;
-  if (sum_blocks >= (int64_t(1) << 31) || fix_blocks >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
-  if (launch_pdl(ss_sum_kernel, dim3(static_cast<unsigned>(sum_blocks)), dim3(SS_WARPS * 32), SS_SUM_SMEM, s, a, nbu,
-                 nbh) !=
-          cudaSuccess ||
+  if (fix_blocks >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  const int64_t units = seg_max + w.maxp;  // per level: segments, then hot pieces
+  const int64_t row_blocks = (static_cast<int64_t>(L) * units + SS_RWARPS - 1) / SS_RWARPS;
+  if (row_blocks >= (int64_t(1) << 31)) return RVQ_ERR_UNSUPPORTED;
+  if (launch_pdl(ss_rowsum_kernel, dim3(static_cast<unsigned>(row_blocks)), dim3(SS_RWARPS * 32), SS_RSMEM, s, a,
+                 units, seg_max) != cudaSuccess ||
       launch_pdl(ss_fix_kernel, dim3(static_cast<unsigned>(fix_blocks)), dim3(SS_WARPS * 32), 0, s, a, hot_max) !=
           cudaSuccess)
     return RVQ_ERR_CUDA;

@@ -26,6 +26,9 @@ def test_reference_arm_prints_one_contract_line():
     assert d["e2e"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"].startswith("tiny")
+    import bench as b
+    import workloads
+    assert d["config"] == json.loads(json.dumps(b.run_config(workloads.WORKLOADS["tiny"], 1)))  # same as the GPU arm
 
 
 def test_traffic_lookup_requires_the_captured_source(tmp_path, monkeypatch):

@@ -79,6 +79,8 @@ def _case(seed, N, L, K, H, zipf=None):
     (1, 2, 7, 4, None),           # a single row
     (40000, 2, 49151, 20, 1.05),  # sorted: the largest K, many empty ids, two column slices
     (70000, 3, 300, 8, None),     # sorted: several histogram chunks, ragged last chunk
+    (5000, 3, 300, 1100, 1.1),    # sorted: two 1024-column passes per segment, the second ragged
+    (3000, 2, 200, 2048, None),   # sorted: two full passes
 ])
 def test_embed_backward_matches_oracle(N, L, K, H, zipf, sort):
     ids, g = _case(N * 7 + L, N, L, K, H, zipf)

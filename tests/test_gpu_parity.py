@@ -138,6 +138,8 @@ EDGE = [
     (200, 64, 4, 4096, "f32", "bf16"),
     (1000, 192, 3, 1000, "bf16", "f32"),
     (4100, 64, 2, 33, "f32", "f32"),
+    (130, 4096, 2, 300, "bf16", "f32"),     # the widest rows the encode takes (streamed, per level)
+    (40, 4096, 1, 17, "f32", "bf16"),
 ]
 
 
