@@ -75,6 +75,10 @@ def test_host_argument_checks(lib):
     assert L.rvq_encode_levels_per_launch(100, 1024, 4, 8192, None) == -1    # no output
     assert L.rvq_encode_levels_per_launch(100, 1000, 4, 8192, ctypes.byref(lv)) == -2   # D % 64
     assert L.rvq_encode_levels_per_launch(100, 1024, 65, 8192, ctypes.byref(lv)) == -2  # L > 64
+    off, slots = ctypes.c_size_t(0), ctypes.c_int32(0)
+    assert L.rvq_encode_candidate_layout(100, 1024, 4, 8192, None, ctypes.byref(slots)) == -1
+    assert L.rvq_encode_candidate_layout(-1, 1024, 4, 8192, ctypes.byref(off), ctypes.byref(slots)) == -1
+    assert L.rvq_encode_candidate_layout(100, 96, 4, 8192, ctypes.byref(off), ctypes.byref(slots)) == -2
     eb = L.rvq_embed_backward
     assert eb(16, 0, 2, 8, 64, 16, 16, None, None) == 0                        # N = 0: no-op
     assert eb(None, 5, 2, 8, 64, 16, 16, None, None) == -1                     # no ids
