@@ -323,16 +323,19 @@ def encode_figures(name, dev, peaks, flush_l2, reps=3):
     stream = torch.cuda.current_stream(dev)
     for _ in range(2):
         tok.encode(x, offsets=off, out=out, fallbacks=fb)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ts = []
     for _ in range(reps):
         fb.zero_()
         flush_l2()
         e0.record(stream)
-        tok.encode(x, offsets=off, out=out, fallbacks=fb, check=False)
+        tok.encode(x, offsets=off, out=out, fallbacks=fb, status=status, check=False)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ts.append(e0.elapsed_time(e1))
+    if int(status.item()) != 0:
+        raise mvt.RVQError(int(status.item()), f"rvq_encode ({name}, device)")
     ms = statistics.median(ts)
     tflops = 2.0 * N * K * D * L / (ms / 1e3) / 1e12
     sus = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
