@@ -337,6 +337,25 @@ def encode_figures(name, dev, peaks, flush_l2, reps=3):
     if int(status.item()) != 0:
         raise mvt.RVQError(int(status.item()), f"rvq_encode ({name}, device)")
     ms = statistics.median(ts)
+    # the decode of the ids just produced (gather-sum back to fp32 features)
+    rec = torch.empty((N, D), dtype=torch.float32, device=dev)
+    td = []
+    for _ in range(reps):
+        flush_l2()
+        e0.record(stream)
+        tok.decode(out["ids"], out=rec, status=status, check=False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        td.append(e0.elapsed_time(e1))
+    if int(status.item()) != 0:
+        raise mvt.RVQError(int(status.item()), f"rvq_decode ({name}, device)")
+    dms = statistics.median(td)
+    ids_h = out["ids"].cpu().numpy()
+    s_cb = 2 if spec.cb_dtype == "bf16" else 4
+    rows_used = sum(int(np.unique(ids_h[:, l]).size) for l in range(L))
+    dbytes = N * L * 4 + rows_used * D * s_cb + N * D * 4
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    del rec
     tflops = 2.0 * N * K * D * L / (ms / 1e3) / 1e12
     sus = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
@@ -344,6 +363,8 @@ def encode_figures(name, dev, peaks, flush_l2, reps=3):
     return {"workload": workload_label(spec), "N": N, "D": D, "L": L, "K": K, "encode_ms": ms,
             "Mtok_per_s": N / (ms / 1e3) / 1e6, "tflops": tflops, "frac_sustained": tflops / sus,
             "frac_burst": tflops / burst, "fallbacks_per_level": fb.cpu().tolist(),
+            "decode_ms": dms, "decode_algorithmic_bytes": dbytes,
+            "decode_frac_hbm": dbytes / (dms / 1e3) / 1e9 / hbm,
             "kernel": "encode_flow_kernel" if lpl > 1 else "dist_topk_kernel per level",
             "timing": f"median of {reps} calls, L2 flushed before each"}
 
