@@ -150,80 +150,111 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const int32_t
   if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
 }
 
-// The same with the number of levels known at compile time (LC <= 16): a warp walks rows
-// w, w + W, ... of one slice with all LC gathers of a row in flight at once, and fetches the next
-// row's ids while the current row's gathers are outstanding, so every L2 round trip a warp
-// waits for carries a full row of gathers.  Three blocks per SM leave each thread enough
-// registers to keep all LC gathers of a row live without spilling.
-template <bool CB_BF16, int VEC, int LC>
+// The same with the number of levels known at compile time (LC <= 16): a warp walks rows of one
+// slice with all LC gathers of a row in flight at once, and fetches the next rows' ids while the
+// current row's gathers are outstanding, so every L2 round trip a warp waits for carries a full row
+// of gathers.  RPW rows share a warp (32 / RPW lanes per row), which narrows the slice to
+// 32 / RPW * VEC columns: the launch picks RPW so that the slice's live codebook columns (L * K *
+// slice * element size bytes) stay within kDecodeLiveBytes of L2.  Three blocks per SM leave each
+// thread enough registers to keep all LC gathers of a row live without spilling.
+constexpr int64_t kDecodeLiveBytes = int64_t(64) << 20;
+
+template <bool CB_BF16, int VEC, int LC, int RPW>
 __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeBlocksPerSm) decode_fixed_kernel(const int32_t *__restrict__ ids,
                                                                            int64_t N, const void *__restrict__ cb,
                                                                            int K, int D, float *__restrict__ recon,
                                                                            int32_t *status) {
+  constexpr int LPR = 32 / RPW;  // lanes per row
+  static_assert(LC <= LPR, "a row's ids are held by the lanes of its own group");
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kDecodeWarps;
-  int64_t n = static_cast<int64_t>(blockIdx.x) * kDecodeWarps + (threadIdx.x >> 5);
-  if (n >= N) return;  // whole warp
-  const int col = blockIdx.y * (32 * VEC) + lane * VEC;
+  const int grp = lane / LPR, gl = lane % LPR;
+  const unsigned full = 0xffffffffu;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kDecodeWarps * RPW;
+  int64_t base = (static_cast<int64_t>(blockIdx.x) * kDecodeWarps + (threadIdx.x >> 5)) * RPW;
+  if (base >= N) return;  // whole warp
+  const int col = blockIdx.y * (LPR * VEC) + gl * VEC;
   const bool active = col < D;
   const int colc = active ? col : 0;
-  int myid = lane < LC ? __ldg(ids + n * LC + lane) : 0;
+  int64_t n = base + grp;
+  int myid = (gl < LC && n < N) ? __ldg(ids + n * LC + gl) : 0;
   bool bad = false;
   while (true) {
+    const bool live = n < N;  // the warp's last rows may lie past N (never stored)
     Gather<CB_BF16, VEC> g[LC];
     bool use[LC];
 #pragma unroll
     for (int l = 0; l < LC; ++l) {
-      const int id = __shfl_sync(0xffffffffu, myid, l);
-      const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(K);
-      bad |= !ok;
-      use[l] = ok;
-      g[l].load(cb, (static_cast<int64_t>(l) * K + (ok ? id : 0)) * D + colc);
+      const int id = __shfl_sync(full, myid, grp * LPR + l);
+      const bool in_range = static_cast<unsigned>(id) < static_cast<unsigned>(K);
+      bad |= live && !in_range;
+      use[l] = live && in_range;
+      g[l].load(cb, (static_cast<int64_t>(l) * K + (use[l] ? id : 0)) * D + colc);
     }
-    const int64_t nn = n + stride;
-    const int nextid = (lane < LC && nn < N) ? __ldg(ids + nn * LC + lane) : 0;
+    const int64_t nbase = base + step;
+    const int64_t nn = nbase + grp;
+    const int nextid = (gl < LC && nn < N) ? __ldg(ids + nn * LC + gl) : 0;
     float acc[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
 #pragma unroll
     for (int l = 0; l < LC; ++l)
       if (use[l]) g[l].add_to(acc);
-    if (active) {
+    if (active && live) {
       float4 *dst = reinterpret_cast<float4 *>(recon + n * D + col);
 #pragma unroll
       for (int k = 0; k < VEC; k += 4) __stcs(dst + k / 4, make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]));
     }
-    if (nn >= N) break;
+    if (nbase >= N) break;
+    base = nbase;
     n = nn;
     myid = nextid;
   }
-  if (bad && lane == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
+  if (bad && gl == 0 && blockIdx.y == 0) set_status(status, RVQ_ERR_ID_RANGE);
 }
 
-template <bool CB_BF16, int VEC, int LC>
+template <bool CB_BF16, int VEC, int LC, int RPW>
 cudaError_t launch_fixed(const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon, int32_t *status,
                          cudaStream_t s) {
-  // per slice, enough blocks to fill every SM at the kernel's occupancy (6 blocks of 8 warps);
-  // each warp then walks rows with a stride of the slice's warp count
+  // per slice, enough blocks to fill every SM at the kernel's occupancy; each warp then walks rows
+  // with a stride of the slice's rows per sweep
   int sms = 0;
   if (device_sm_count(&sms) != RVQ_OK) return cudaErrorUnknown;
-  const int64_t gx = std::min<int64_t>((N + kDecodeWarps - 1) / kDecodeWarps, static_cast<int64_t>(sms) * kDecodeBlocksPerSm);
-  const int gy = (D + 32 * VEC - 1) / (32 * VEC);
+  const int64_t warps = (N + RPW - 1) / RPW;
+  const int64_t gx = std::min<int64_t>((warps + kDecodeWarps - 1) / kDecodeWarps,
+                                       static_cast<int64_t>(sms) * kDecodeBlocksPerSm);
+  const int width = 32 / RPW * VEC;
+  const int gy = (D + width - 1) / width;
   if (gx > 0x7FFFFFFFLL || gy > 65535) return cudaErrorInvalidValue;
-  return launch_pdl(decode_fixed_kernel<CB_BF16, VEC, LC>, dim3(static_cast<unsigned>(gx), gy),
+  return launch_pdl(decode_fixed_kernel<CB_BF16, VEC, LC, RPW>, dim3(static_cast<unsigned>(gx), gy),
                     dim3(kDecodeWarps * 32), 0, s, ids, N, cb, K, D, recon, status);
 }
 
+// Rows per warp for a decode of L levels of K codewords of elem_bytes each: the widest slice whose
+// live codebook columns fit kDecodeLiveBytes, or the narrowest one whose lane groups still hold a
+// row's L ids.
+inline int decode_rows_per_warp(int L, int K, int VEC, int elem_bytes) {
+  int rpw = 1;
+  while (rpw < 4 && L <= 32 / (2 * rpw) &&
+         static_cast<int64_t>(L) * K * (32 / rpw * VEC) * elem_bytes > kDecodeLiveBytes)
+    rpw *= 2;
+  return rpw;
+}
+
 template <bool CB_BF16, int VEC, int LC = 1>
-cudaError_t dispatch_fixed(int L, const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon,
+cudaError_t dispatch_fixed(int L, int rpw, const int32_t *ids, int64_t N, const void *cb, int K, int D, float *recon,
                            int32_t *status, cudaStream_t s) {
   if constexpr (LC > 16) {
     return cudaErrorInvalidValue;
   } else {
-    if (L == LC) return launch_fixed<CB_BF16, VEC, LC>(ids, N, cb, K, D, recon, status, s);
-    return dispatch_fixed<CB_BF16, VEC, LC + 1>(L, ids, N, cb, K, D, recon, status, s);
+    if (L == LC) {
+      if constexpr (LC <= 8)
+        if (rpw == 4) return launch_fixed<CB_BF16, VEC, LC, 4>(ids, N, cb, K, D, recon, status, s);
+      if (rpw == 2) return launch_fixed<CB_BF16, VEC, LC, 2>(ids, N, cb, K, D, recon, status, s);
+      return launch_fixed<CB_BF16, VEC, LC, 1>(ids, N, cb, K, D, recon, status, s);
+    }
+    return dispatch_fixed<CB_BF16, VEC, LC + 1>(L, rpw, ids, N, cb, K, D, recon, status, s);
   }
 }
 
@@ -239,11 +270,14 @@ int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_d
   if (N == 0) return RVQ_OK;
   if (L <= 16) {
     cudaError_t e;
-    if (cb_dtype == RVQ_BF16)
-      e = D % 8 == 0 ? dispatch_fixed<true, 8>(L, ids, N, cb, K, D, recon, status, s)
-                                        : dispatch_fixed<true, 4>(L, ids, N, cb, K, D, recon, status, s);
-    else
-      e = dispatch_fixed<false, 4>(L, ids, N, cb, K, D, recon, status, s);
+    if (cb_dtype == RVQ_BF16) {
+      if (D % 8 == 0)
+        e = dispatch_fixed<true, 8>(L, decode_rows_per_warp(L, K, 8, 2), ids, N, cb, K, D, recon, status, s);
+      else
+        e = dispatch_fixed<true, 4>(L, decode_rows_per_warp(L, K, 4, 2), ids, N, cb, K, D, recon, status, s);
+    } else {
+      e = dispatch_fixed<false, 4>(L, decode_rows_per_warp(L, K, 4, 4), ids, N, cb, K, D, recon, status, s);
+    }
     note_launch();
     return e == cudaSuccess ? RVQ_OK : e == cudaErrorInvalidValue ? RVQ_ERR_UNSUPPORTED : RVQ_ERR_CUDA;
   }

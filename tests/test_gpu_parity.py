@@ -431,3 +431,50 @@ def test_bf16_decode_whole_slices(N, L, K, D):
     others = np.ones(N, bool)
     others[[0, N // 2]] = False
     assert np.array_equal(rec2[others], rec.cpu().numpy()[others])
+
+
+@pytest.mark.parametrize("L,K,D,dt", [
+    (4, 65536, 256, "f32"),   # 128-column slices would hold 128 MiB of codebook: two rows per warp
+    (8, 65536, 128, "f32"),   # four rows per warp (32-column slices)
+    (8, 65536, 256, "bf16"),  # four rows per warp, 16-byte bf16 gathers
+    (12, 32768, 132, "bf16"),  # D % 8 != 0: 8-byte gathers, two rows per warp
+])
+def test_decode_narrow_slices(L, K, D, dt):
+    """Codebooks whose live columns outgrow L2 are decoded in narrower slices with several rows per
+    warp: every row against the oracle at ragged counts (fewer rows than a warp holds included),
+    and out-of-range ids in rows held by different lane groups set the status and drop only
+    their own level.  Called through rvq_decode itself (D % 64 != 0 is a decode-only width)."""
+    rng = np.random.Generator(np.random.PCG64([L, K, D, 11]))
+    C = rng.standard_normal((L, K, D), dtype=np.float32)
+    if dt == "bf16":
+        C = workloads.round_bf16(C)
+    Cd = dev(C, dt)
+    code = mvt.RVQ_BF16 if dt == "bf16" else mvt.RVQ_F32
+
+    def decode(ids):
+        N = ids.shape[0]
+        rec = torch.empty((N, D), dtype=torch.float32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        assert mvt.rvq_decode(torch.from_numpy(ids).cuda(), N, L, Cd, code, K, D, rec, st) == 0
+        torch.cuda.synchronize()
+        return rec.cpu().numpy(), int(st.item())
+
+    for N in (1, 3, 5003):
+        ids = rng.integers(0, K, size=(N, L)).astype(np.int32)
+        rec, st = decode(ids)
+        assert st == 0
+        parity.check_recon(None, C, np.arange(N), ids, recon_gpu=rec)
+    bad = ids.copy()
+    hit = [1, 2, N - 1]
+    bad[1, L - 1] = K
+    bad[2, 0] = -1
+    bad[N - 1, L // 2] = 1 << 30
+    rec2, st = decode(bad)
+    assert st == -5
+    keep = (bad >= 0) & (bad < K)
+    for n in hit:
+        want = sum(C[l, bad[n, l]].astype(np.float64) for l in range(L) if keep[n, l])
+        assert np.allclose(rec2[n], want, rtol=1e-5, atol=1e-5)
+    others = np.ones(N, bool)
+    others[hit] = False
+    assert np.array_equal(rec2[others], rec[others])
