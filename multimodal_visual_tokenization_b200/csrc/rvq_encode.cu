@@ -19,9 +19,13 @@
 //    row tile rt) start as soon as the certificate warps have settled level l-1 of rt (counter
 //    cert_done[l-1][rt]); the certificate warps take (l, rt) once all its chunks are written
 //    (chunk_done[l][rt]).  Per CTA: a TMA producer warp, an MMA-issuer warp, a norm-split warp,
-//    8 epilogue warps and 4 (D = 1024) or 3 (D = 256) certificate warps.  Rows the certificate
-//    cannot settle get an exact scan of all K codewords, cut into slices any certificate warp may
-//    run.  Every wait is bounded (status RVQ_ERR_TIMEOUT when nothing moved for two seconds).
+//    4 epilogue + 4 certificate warps (D in (512, 1024]) or 8 + 3 (D in (128, 256]).  For D in
+//    (512, 1024] and batches of at least kPairMinRows rows the CTAs run as pairs (2-CTA clusters,
+//    tcgen05 cta_group::2): each CTA loads its own 128 rows and half of every 256-codeword tile,
+//    the leader issues M = 256 MMAs, and each CTA's TMEM holds its own rows' accumulators, so an
+//    SM streams 32 KB instead of 48 KB per K step.  Rows the certificate cannot settle get an
+//    exact scan of all K codewords, cut into slices any certificate warp may run.  Every wait is
+//    bounded (status RVQ_ERR_TIMEOUT when nothing moved for two seconds).
 //  * other widths (and RVQ_PERSISTENT=0): per level, dist_topk_kernel (persistent GEMM + top-8 over
 //    contiguous ranges of (row tile, codeword tile) units, 4 or 8 epilogue warps), then
 //    rescore_fast_kernel / rescore_kernel (certificate, one warp per row) and
@@ -1409,12 +1413,29 @@ struct FlowCfg {
   static constexpr int CERT_WARPS = RW - __builtin_popcount(SKIP);
 };
 
-template <int EPI, int RW, int SKIP, bool CB_BF16, bool X_BF16, int NCH>
+// Shared memory of the all-levels kernel.  A CTA of a pair (cta_group::2) loads its own 128 rows
+// and half of each 256-codeword tile, so a stage is A 16 KB + B 16 KB and six stages fit where
+// four single-CTA stages of 48 KB do.
+template <int EPI, bool PAIR>
+struct FlowMem : GemmCfg<EPI> {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // codeword rows of a tile this CTA loads
+  static constexpr int STAGE = A_BYTES + B_ROWS * BK * 2;
+  static constexpr int NSTAGE = PAIR ? 6 : GemmCfg<EPI>::NSTAGE;
+  static constexpr int AUG_A_OFF = NSTAGE * STAGE;
+  static constexpr int AUG_B_OFF = AUG_A_OFF + AUG_A_BYTES;
+  static constexpr int MERGE_OFF = AUG_B_OFF + 2 * AUG_B_BYTES;
+  static constexpr int BAR_OFF = MERGE_OFF + (GemmCfg<EPI>::GROUPS - 1) * BM * TOPK * 8;
+  static constexpr int SMEM = BAR_OFF + 512 + 1024;
+  static_assert(SMEM <= 232448, "dynamic shared memory above the 227 KB per-block limit");
+  static_assert(!PAIR || GemmCfg<EPI>::GROUPS == 1, "pairs run one epilogue column group");
+};
+
+template <int EPI, int RW, int SKIP, bool CB_BF16, bool X_BF16, int NCH, bool PAIR>
 __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     encode_flow_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB3, const GemmArgs a, const RowArgs r0,
                        const FlowArgs fa) {
-  using C = GemmCfg<EPI>;
+  using C = FlowMem<EPI, PAIR>;
   constexpr int NSTAGE = C::NSTAGE;
   constexpr int CERT0 = FlowCfg<EPI, RW, SKIP>::CERT0;
   constexpr int CW = FlowCfg<EPI, RW, SKIP>::CERT_WARPS;
@@ -1441,7 +1462,14 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
   const int KB = a.D / BK;
   const uint32_t G = gridDim.x;
   const int64_t RT = fa.RT;
-  const int64_t total_chunks = static_cast<int64_t>(fa.L) * RT * fa.NC;
+  // Chunks are walked by CTAs, or by CTA pairs over 256-row units (unit u holds row tiles 2u and
+  // 2u+1, the second of which may lie past the last row tile).
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0: the pair's leader (issues the MMAs)
+  const uint32_t GW = PAIR ? G / 2 : G;                  // chunk walkers
+  const uint32_t wid = PAIR ? blockIdx.x / 2 : blockIdx.x;
+  const int64_t RU = PAIR ? (RT + 1) / 2 : RT;           // row units
+  const int64_t total_chunks = static_cast<int64_t>(fa.L) * RU * fa.NC;
+  auto own_tile = [&](int64_t ru) -> int64_t { return PAIR ? 2 * ru + rank : ru; };
   uint32_t *ex_rows = fa.ctr;
   uint32_t *ex_next = fa.ctr + 1;
   uint32_t *settled = fa.ctr + 2;
@@ -1452,7 +1480,7 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
   };
   // First codeword tile this CTA visits in a chunk of cnt tiles: CTAs spread their starting
   // points over the chunk so they do not all stream the same codeword tile at the same time.
-  auto chunk_rot = [&](int cnt) -> int { return static_cast<int>((static_cast<int64_t>(blockIdx.x) * cnt) / G); };
+  auto chunk_rot = [&](int cnt) -> int { return static_cast<int>((static_cast<int64_t>(wid) * cnt) / GW); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -1461,8 +1489,8 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EPI_THREADS);
-      mbar_init(&afull[b], 32);
+      mbar_init(&tempty[b], (PAIR ? 2 : 1) * C::EPI_THREADS);  // a pair's epilogues both release the leader's
+      mbar_init(&afull[b], PAIR ? 64 : 32);
     }
     mbar_init(mready, C::EPI_THREADS - 128 > 0 ? C::EPI_THREADS - 128 : 1);
     mbar_init(mdone, 128);
@@ -1479,13 +1507,25 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
   }
   fence_proxy_async_smem();
   if (warp == C::ISSUER) {
-    tmem_alloc(tmem_holder, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_holder, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the leader's barriers, as seen from either CTA of a pair
+  const uint32_t full_l = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+  const uint32_t tempty_l = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
+  const uint32_t afull_l = PAIR ? mapa_shared(smem_u32(afull), 0) : 0u;
 
   int p_s = 0;  // producer ring position, kept for the teardown
   uint32_t p_ph = 0;
@@ -1498,11 +1538,11 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB3);
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+      for (int64_t t = wid; t < total_chunks && ok; t += GW) {
         const int j = static_cast<int>(t % fa.NC);
-        const int64_t rt = (t / fa.NC) % RT;
-        const int l = static_cast<int>(t / (fa.NC * RT));
-        if (l > 0) {
+        const int64_t rt = own_tile((t / fa.NC) % RU);
+        const int l = static_cast<int>(t / (fa.NC * RU));
+        if (l > 0 && rt < RT) {  // a pair's second tile past the last row tile holds no rows
           if (!wait_count(fa.cert_done + (l - 1) * RT + rt, tile_rows(rt), progress, abort_flag)) {
             ok = false;
             break;
@@ -1519,10 +1559,17 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&full[p_s], C::STAGE);
             uint8_t *sa = smem + p_s * C::STAGE;
-            tma_load_2d(mA, &full[p_s], sa, kb * BK, static_cast<int32_t>(rt * BM));
-            tma_load_3d(&tmB3, &full[p_s], sa + A_BYTES, kb * BK, ct * BN, l);
+            if constexpr (PAIR) {  // both CTAs' bytes complete the leader's barrier
+              if (rank == 0) mbar_arrive_expect_tx(&full[p_s], 2 * C::STAGE);
+              tma_load_2d_pair(mA, full_l + p_s * 8, sa, kb * BK, static_cast<int32_t>(rt * BM));
+              tma_load_3d_pair(&tmB3, full_l + p_s * 8, sa + A_BYTES, kb * BK,
+                               ct * BN + static_cast<int32_t>(rank) * C::B_ROWS, l);
+            } else {
+              mbar_arrive_expect_tx(&full[p_s], C::STAGE);
+              tma_load_2d(mA, &full[p_s], sa, kb * BK, static_cast<int32_t>(rt * BM));
+              tma_load_3d(&tmB3, &full[p_s], sa + A_BYTES, kb * BK, ct * BN, l);
+            }
             ++p_issued;
             if (++p_s == NSTAGE) {
               p_s = 0;
@@ -1540,19 +1587,21 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     // ------------------------------------------------------------ norm split -> B_aug tiles
     int64_t i = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+    // this CTA's codeword rows of a tile in groups of 8 (a pair's CTA holds half the tile)
+    const bool writer = lane < C::B_ROWS / 8;
+    for (int64_t t = wid; t < total_chunks && ok; t += GW) {
       const int j = static_cast<int>(t % fa.NC);
-      const int l = static_cast<int>(t / (fa.NC * RT));
+      const int l = static_cast<int>(t / (fa.NC * RU));
       const float *norms_l = fa.norms + static_cast<int64_t>(l) * a.K;
       const int ct0 = j * fa.S, cnt = min(a.Tc, ct0 + fa.S) - ct0;
       const int rot = chunk_rot(cnt);
       for (int k = 0; k < cnt; ++k, ++i) {
         const int ct = ct0 + (rot + k) % cnt;
         const int slot = static_cast<int>(i & 1);
-        const int c0 = ct * BN + lane * 8;
+        const int c0 = ct * BN + static_cast<int>(rank) * C::B_ROWS + lane * 8;
         float hv[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) hv[q] = c0 + q < a.K ? 0.5f * __ldg(norms_l + c0 + q) : 0.f;
+        for (int q = 0; q < 8; ++q) hv[q] = (writer && c0 + q < a.K) ? 0.5f * __ldg(norms_l + c0 + q) : 0.f;
         bool got = i < 2 || mbar_wait(&tfull[slot], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
@@ -1562,6 +1611,7 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
         uint4 *dst = reinterpret_cast<uint4 *>(aug_b + slot * AUG_B_BYTES + lane * 128);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
+          if (!writer) break;
           uint16_t h1, h2 = 0, h3 = 0;
           if (c0 + q < a.K) {
             h1 = bf16_bits_rn(hv[q]);
@@ -1575,7 +1625,10 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
           dst[q] = make_uint4(h1 | (static_cast<uint32_t>(h2) << 16), h3, 0, 0);
         }
         fence_proxy_async_smem();
-        mbar_arrive(&afull[slot]);
+        if constexpr (PAIR)
+          mbar_arrive_cluster(afull_l + slot * 8);
+        else
+          mbar_arrive(&afull[slot]);
       }
     }
     if (!ok) {
@@ -1583,16 +1636,16 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
       set_status(a.status, RVQ_ERR_TIMEOUT);
     }
   } else if (warp == C::ISSUER) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_main = idesc_bf16_f32(BM, BN, true);
-      constexpr uint32_t idesc_aug = idesc_bf16_f32(BM, BN, false);
+    // ------------------------------------------------------------ MMA issuer (a pair's leader)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc_main = idesc_bf16_f32(PAIR ? 2 * BM : BM, BN, true);
+      constexpr uint32_t idesc_aug = idesc_bf16_f32(PAIR ? 2 * BM : BM, BN, false);
       const uint64_t adesc_aug = sdesc_k_noswizzle(smem_u32(aug_a), 128, 256);
       int m_s = 0;
       uint32_t m_ph = 0;
       int64_t i = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+      for (int64_t t = wid; t < total_chunks && ok; t += GW) {
         const int j = static_cast<int>(t % fa.NC);
         const int cnt = min(a.Tc, j * fa.S + fa.S) - j * fa.S;
         for (int k = 0; k < cnt && ok; ++k, ++i) {
@@ -1604,7 +1657,11 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
           }
           tc_fence_after();
           const uint32_t dt = tmem_base + static_cast<uint32_t>(buf * BN);
-          umma_f16(dt, adesc_aug, sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128), idesc_aug, 0u);
+          const uint64_t bdesc_aug = sdesc_k_noswizzle(smem_u32(aug_b + buf * AUG_B_BYTES), 128, 128);
+          if constexpr (PAIR)
+            umma_f16_pair(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
+          else
+            umma_f16(dt, adesc_aug, bdesc_aug, idesc_aug, 0u);
           for (int kb = 0; kb < KB; ++kb) {
             if (!mbar_wait(&full[m_s], m_ph, abort_flag)) {
               ok = false;
@@ -1617,16 +1674,25 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / UK; ++k) {
               const uint64_t step = static_cast<uint64_t>(k * UK * 2 / 16);
-              umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
+              if constexpr (PAIR)
+                umma_f16_pair(dt, ad + step, bd + step, idesc_main, 1u);
+              else
+                umma_f16(dt, ad + step, bd + step, idesc_main, 1u);
             }
-            umma_commit(&empty[m_s]);
+            if constexpr (PAIR)
+              umma_commit_pair_both(&empty[m_s]);  // frees the stage in both CTAs
+            else
+              umma_commit(&empty[m_s]);
             if (++m_s == NSTAGE) {
               m_s = 0;
               m_ph ^= 1u;
             }
           }
           if (!ok) break;
-          umma_commit(&tfull[buf]);
+          if constexpr (PAIR)
+            umma_commit_pair_both(&tfull[buf]);  // both CTAs' epilogues may read their TMEM rows
+          else
+            umma_commit(&tfull[buf]);
         }
       }
       if (!ok) {
@@ -1645,10 +1711,11 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     int64_t i = 0;
     uint32_t nflush = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < total_chunks && ok; t += G) {
+    for (int64_t t = wid; t < total_chunks && ok; t += GW) {
       const int j = static_cast<int>(t % fa.NC);
-      const int64_t rt = (t / fa.NC) % RT;
-      const int l = static_cast<int>(t / (fa.NC * RT));
+      const int64_t rt = own_tile((t / fa.NC) % RU);
+      const bool rows_here = rt < RT;  // false only for a pair's second tile past the last row tile
+      const int l = static_cast<int>(t / (fa.NC * RU));
 #pragma unroll
       for (int q = 0; q < TOPK; ++q) {
         bd[q] = inf_f();
@@ -1657,7 +1724,8 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
       // slot j of (l-1, rt) must have been read by every certificate task before it is rewritten:
       // the producer already waited for that, so this load (checked at the flush) only orders it
       uint32_t settled_prev = 0xffffffffu;
-      if (grp == 0 && lane == 0 && l > 0) settled_prev = ld_acquire_gpu(fa.cert_done + (l - 1) * RT + rt);
+      if (grp == 0 && lane == 0 && l > 0 && rows_here)
+        settled_prev = ld_acquire_gpu(fa.cert_done + (l - 1) * RT + rt);
       const int ct0 = j * fa.S, cnt = min(a.Tc, ct0 + fa.S) - ct0;
       const int rot = chunk_rot(cnt);
       for (int k = 0; k < cnt; ++k, ++i) {
@@ -1681,7 +1749,10 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
           tmem_ld_wait();
           if (ch == C::CHUNKS - 1) {
             tc_fence_before();
-            mbar_arrive(&tempty[buf]);
+            if constexpr (PAIR)
+              mbar_arrive_cluster(tempty_l + buf * 8);
+            else
+              mbar_arrive(&tempty[buf]);
           }
           const int c0 = col0 + ct0;
           float d[32];
@@ -1733,7 +1804,7 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
         }
       }
       ++nflush;
-      if (grp == 0) {
+      if (grp == 0 && rows_here) {
         // the slot is rewritten only after every certificate task of (l-1, rt) has read it
         bool got = true;
         if (lane == 0 && settled_prev < tile_rows(rt))
@@ -1957,12 +2028,16 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
     }
   }
 
-  // no bulk copy or MMA may still be in flight when the block exits
-  if (warp == C::ISSUER && lane == 0) {
-    umma_commit(mma_done);
+  // no bulk copy or MMA may still be in flight when the block exits (a pair's MMAs and bytes are
+  // counted on the leader's barriers, so the leader waits for both CTAs)
+  if (warp == C::ISSUER && lane == 0 && rank == 0) {
+    if constexpr (PAIR)
+      umma_commit_pair(mma_done);
+    else
+      umma_commit(mma_done);
     mbar_wait(mma_done, 0, never);
   }
-  if (warp == C::PRODUCER && lane == 0 && *abort_flag) {
+  if (warp == C::PRODUCER && lane == 0 && *abort_flag && rank == 0) {
     const int64_t pending = p_issued < NSTAGE ? p_issued : NSTAGE;
     for (int64_t jj = 0; jj < pending; ++jj) {
       int back = p_s - 1 - static_cast<int>(jj);
@@ -1977,10 +2052,14 @@ __global__ void __launch_bounds__(FlowCfg<EPI, RW, SKIP>::THREADS, 1)
   tc_fence_before();
   __syncwarp();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer may signal this CTA's barriers until both are done
   tc_fence_after();
   if (warp == C::ISSUER) {
     __syncwarp();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -1999,7 +2078,16 @@ struct Plan {
   int RPT;        // rows per certificate task
   int NS, slice;  // exact-scan slices per queued row, codewords per slice
   int Gf;         // CTAs of the flow launch (one per SM)
+  bool fpair;     // the flow launch runs CTA pairs (cta_group::2) over 256-row units
 };
+
+// Smallest batch that the all-levels kernel runs as CTA pairs.  Pairs halve each SM's codeword
+// tile traffic and draw less power, which pays under the power cap of a long launch (2^20 rows
+// of D = 1024, L = 8, K = 16384: 222 vs 238 ms; 206181 rows, L = 8: 45 vs 46.5 ms); a launch
+// short enough to run at the boost clock (4096 rows) is faster with single CTAs.
+constexpr int64_t kPairMinRows = 65536;
+
+inline bool flow_pairs_fit(int grid);
 
 // RVQ_PERSISTENT=0 keeps the per-level launches for every width (tuning / comparison knob).
 inline bool persistent_enabled() {
@@ -2041,10 +2129,16 @@ inline Plan make_plan(int64_t N, int K, int D, int L, int sms) {
   p.flow = D <= 1024 && (nch == 2 || nch == 8) && persistent_enabled() &&
            static_cast<uint64_t>(N) * static_cast<uint64_t>(L) < (uint64_t(1) << 32);
   p.NC = p.S = p.RPT = p.NS = p.slice = p.Gf = 0;
+  p.fpair = false;
   if (p.flow) {
     p.Gf = sms;
-    // enough chunks per level to keep every CTA busy and finish a row tile soon after it starts
-    int nc = static_cast<int>(std::min<int64_t>(MAX_SLOTS, std::max<int64_t>(1, (4 * p.Gf + p.RT - 1) / p.RT)));
+    // CTA pairs halve the codeword-tile traffic of each SM (each CTA of a pair loads half of a
+    // tile); they pay on batches long enough to run under the power cap
+    p.fpair = nch == 8 && N >= kPairMinRows && flow_pairs_fit(p.Gf);
+    const int64_t units = p.fpair ? (p.RT + 1) / 2 : p.RT;
+    const int64_t walkers = p.fpair ? p.Gf / 2 : p.Gf;
+    // enough chunks per level to keep every walker busy and finish a row tile soon after it starts
+    int nc = static_cast<int>(std::min<int64_t>(MAX_SLOTS, std::max<int64_t>(1, (4 * walkers + units - 1) / units)));
     nc = std::min(nc, p.Tc);
     p.S = (p.Tc + nc - 1) / nc;
     p.NC = (p.Tc + p.S - 1) / p.S;  // no empty chunk
@@ -2185,10 +2279,10 @@ inline cudaError_t launch_gemm_t(int groups, cudaStream_t s, const CUtensorMap &
 // All-levels dataflow encode, instantiated for 2 (D in (128, 256]) and 8 (D in (512, 1024])
 // float4 row chunks.
 
-template <int EPI, int RW, int SK, bool CB, bool XB, int NCH>
+template <int EPI, int RW, int SK, bool CB, bool XB, int NCH, bool PAIR = false>
 inline bool set_flow_attr() {
-  return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, SK, CB, XB, NCH>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<EPI>::SMEM) == cudaSuccess;
+  return cudaFuncSetAttribute(encode_flow_kernel<EPI, RW, SK, CB, XB, NCH, PAIR>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, FlowMem<EPI, PAIR>::SMEM) == cudaSuccess;
 }
 
 inline bool flow_attrs_ready() {
@@ -2199,33 +2293,73 @@ inline bool flow_attrs_ready() {
     constexpr int EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW, SN = FLOW_SKIP_NARROW;
     ok = set_flow_attr<EW, RWD, SW, false, false, 8>() && set_flow_attr<EW, RWD, SW, false, true, 8>() &&
          set_flow_attr<EW, RWD, SW, true, false, 8>() && set_flow_attr<EW, RWD, SW, true, true, 8>() &&
+         set_flow_attr<EW, RWD, SW, false, false, 8, true>() && set_flow_attr<EW, RWD, SW, false, true, 8, true>() &&
+         set_flow_attr<EW, RWD, SW, true, false, 8, true>() && set_flow_attr<EW, RWD, SW, true, true, 8, true>() &&
          set_flow_attr<EN, RN, SN, false, false, 2>() && set_flow_attr<EN, RN, SN, false, true, 2>() &&
          set_flow_attr<EN, RN, SN, true, false, 2>() && set_flow_attr<EN, RN, SN, true, true, 2>();
   });
   return ok;
 }
 
-template <int EPI, int RW, int SK, bool CB, bool XB, int NCH>
-inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tmA0, const CUtensorMap &tmA,
-                                 const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(FlowCfg<EPI, RW, SK>::THREADS);
-  cfg.dynamicSmemBytes = GemmCfg<EPI>::SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+template <int EPI, int RW, int SK, bool PAIR>
+inline void flow_launch_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute (&attr)[2], int grid, cudaStream_t s) {
+  *cfg = {};
+  cfg->gridDim = dim3(grid);
+  cfg->blockDim = dim3(FlowCfg<EPI, RW, SK>::THREADS);
+  cfg->dynamicSmemBytes = FlowMem<EPI, PAIR>::SMEM;
+  cfg->stream = s;
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: CTAs wait on one another's counters
   attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, SK, CB, XB, NCH>, tmA0, tmA, tmB3, ga, ra, fa);
+  attr[1].id = cudaLaunchAttributeClusterDimension;  // CTA pairs: clusters of two
+  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg->attrs = attr;
+  cfg->numAttrs = PAIR ? 2 : 1;
 }
 
-inline cudaError_t launch_flow(int nch, bool cb_bf16, bool x_bf16, int grid, cudaStream_t s, const CUtensorMap &tmA0,
-                               const CUtensorMap &tmA, const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra,
-                               const FlowArgs &fa) {
+// Whether `grid` CTAs of the pair kernel for D in (512, 1024] can all be resident as 2-CTA clusters.
+inline bool flow_pairs_fit(int grid) {
+  static std::once_flag once;
+  static int clusters = 0;
+  std::call_once(once, [] {
+    if (!flow_attrs_ready()) return;
+    constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, SW = FLOW_SKIP_WIDE;
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[2];
+    flow_launch_config<EW, RWD, SW, true>(&cfg, attr, 2, nullptr);
+    cfg.numAttrs = 1;  // the occupancy query takes the cluster shape alone
+    cfg.attrs = attr + 1;
+    if (cudaOccupancyMaxActiveClusters(&clusters, encode_flow_kernel<EW, RWD, SW, true, true, 8, true>, &cfg) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      clusters = 0;
+    }
+  });
+  return grid % 2 == 0 && clusters >= grid / 2;
+}
+
+template <int EPI, int RW, int SK, bool CB, bool XB, int NCH, bool PAIR = false>
+inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tmA0, const CUtensorMap &tmA,
+                                 const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  flow_launch_config<EPI, RW, SK, PAIR>(&cfg, attr, grid, s);
+  return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, SK, CB, XB, NCH, PAIR>, tmA0, tmA, tmB3, ga, ra, fa);
+}
+
+inline cudaError_t launch_flow(int nch, bool pair, bool cb_bf16, bool x_bf16, int grid, cudaStream_t s,
+                               const CUtensorMap &tmA0, const CUtensorMap &tmA, const CUtensorMap &tmB3,
+                               const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
   constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, SW = FLOW_SKIP_WIDE;
   constexpr int EN = FLOW_EPI_NARROW, RN = FLOW_RW_NARROW, SN = FLOW_SKIP_NARROW;
+  if (pair) {
+    if (nch != 8) return cudaErrorInvalidValue;
+    if (cb_bf16) return x_bf16 ? launch_flow_t<EW, RWD, SW, true, true, 8, true>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                               : launch_flow_t<EW, RWD, SW, true, false, 8, true>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+    return x_bf16 ? launch_flow_t<EW, RWD, SW, false, true, 8, true>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
+                  : launch_flow_t<EW, RWD, SW, false, false, 8, true>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
+  }
   if (nch == 2) {
     if (cb_bf16) return x_bf16 ? launch_flow_t<EN, RN, SN, true, true, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa)
                                : launch_flow_t<EN, RN, SN, true, false, 2>(grid, s, tmA0, tmA, tmB3, ga, ra, fa);
@@ -2359,7 +2493,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   if (all_levels) {
     if (!flow_attrs_ready()) return RVQ_ERR_CUDA;
     CUtensorMap tmB3;
-    if (!make_map3(&tmB3, op, L, K, D, BN)) return RVQ_ERR_CUDA;
+    if (!make_map3(&tmB3, op, L, K, D, p.fpair ? BN / 2 : BN)) return RVQ_ERR_CUDA;
     if (cudaMemsetAsync(fb_count, 0, w.sync_end - w.fb_count, s) != cudaSuccess) return RVQ_ERR_CUDA;
     uint8_t *sync = ws + w.sync;
     GemmArgs ga;
@@ -2418,7 +2552,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
     fa.norms = norms;
     fa.level_stats = level_stats;
     profile_begin(s);
-    const cudaError_t fe = launch_flow(nch, cb_dtype == RVQ_BF16, f_dtype == RVQ_BF16, p.Gf, s,
+    const cudaError_t fe = launch_flow(nch, p.fpair, cb_dtype == RVQ_BF16, f_dtype == RVQ_BF16, p.Gf, s,
                                        x_is_operand ? tmX : tmA, tmA, tmB3, ga, r0, fa);
     profile_end(s, L);
     note_launch();

@@ -95,6 +95,23 @@ def test_offline_sampled():
     assert (ids[:, 0] == g["planted"][:, 0]).mean() > 0.999   # mixture centre recovered
 
 
+def test_pairs_ragged_last_unit():
+    """A batch long enough for CTA pairs with an odd number of 128-row tiles (the last pair's
+    second tile holds no rows) and a ragged last codeword tile: sampled rows plus every row of the
+    last two row tiles against the oracle, properties on all rows."""
+    N, D, L, K = 65636, 1024, 3, 700
+    rng = np.random.Generator(np.random.PCG64(4242))
+    C = np.stack([rng.standard_normal((K, D), dtype=np.float32) * np.float32(0.5 ** l) for l in range(L)])
+    planted = rng.integers(0, K, size=(N, L)).astype(np.int32)
+    x = sum(C[l][planted[:, l]] for l in range(L)) + rng.standard_normal((N, D), dtype=np.float32) * np.float32(0.05)
+    x = workloads.round_bf16(x)
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32")
+    rows = np.union1d(workloads.sample_rows(N, 4096, seed=9), np.arange(N - 100 - 128, N))
+    rep = full_check(x, C, ids, res, rec, rows)
+    print("pairs ragged", rep, "fallbacks", fb.tolist())
+    assert (ids[:, 0] == planted[:, 0]).all()
+
+
 def test_detok_decode_and_round_trip():
     g = workloads.generate("detok")
     C, want = g["codebooks"], g["planted"]
