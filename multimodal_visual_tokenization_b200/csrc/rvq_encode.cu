@@ -14,8 +14,8 @@
 // warps read it with tcgen05.ld (one TMEM lane = one row) and keep a running top-8 (d~, id) per
 // row; the distance matrix never leaves the SM.
 //
-//  * encode_flow_kernel (D in (128, 256] or (512, 1024]): every level in ONE cooperative launch,
-//    one CTA per SM.  The level loop is a dataflow over 128-row tiles: GEMM chunks of (level l,
+//  * encode_flow_kernel (D in (128, 256] or (512, 1024]): every level in ONE launch with every
+//    CTA resident (cooperative for single CTAs), one CTA per SM.  The level loop is a dataflow over 128-row tiles: GEMM chunks of (level l,
 //    row tile rt) start as soon as the certificate warps have settled level l-1 of rt (counter
 //    cert_done[l-1][rt]); the certificate warps take (l, rt) once all its chunks are written
 //    (chunk_done[l][rt]).  Per CTA: a TMA producer warp, an MMA-issuer warp, a norm-split warp,
@@ -2301,21 +2301,29 @@ inline bool flow_attrs_ready() {
   return ok;
 }
 
+// Single CTAs launch cooperatively (every CTA resident: CTAs wait on one another's counters).
+// Pairs launch as clusters of two without the cooperative attribute (the profiler refuses a
+// cooperative launch with a cluster shape); the plan picks pairs only when the cluster occupancy
+// query puts every cluster on the GPU at once, and a CTA that waits on one that never becomes
+// resident still gives up with RVQ_ERR_TIMEOUT once nothing has moved for two seconds.
 template <int EPI, int RW, int SK, bool PAIR>
-inline void flow_launch_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute (&attr)[2], int grid, cudaStream_t s) {
+inline void flow_launch_config(cudaLaunchConfig_t *cfg, cudaLaunchAttribute (&attr)[1], int grid, cudaStream_t s) {
   *cfg = {};
   cfg->gridDim = dim3(grid);
   cfg->blockDim = dim3(FlowCfg<EPI, RW, SK>::THREADS);
   cfg->dynamicSmemBytes = FlowMem<EPI, PAIR>::SMEM;
   cfg->stream = s;
-  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: CTAs wait on one another's counters
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;  // CTA pairs: clusters of two
-  attr[1].val.clusterDim.x = PAIR ? 2 : 1;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
+  if constexpr (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  }
   cfg->attrs = attr;
-  cfg->numAttrs = PAIR ? 2 : 1;
+  cfg->numAttrs = 1;
 }
 
 // Whether `grid` CTAs of the pair kernel for D in (512, 1024] can all be resident as 2-CTA clusters.
@@ -2326,10 +2334,8 @@ inline bool flow_pairs_fit(int grid) {
     if (!flow_attrs_ready()) return;
     constexpr int EW = FLOW_EPI_WIDE, RWD = FLOW_RW_WIDE, SW = FLOW_SKIP_WIDE;
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     flow_launch_config<EW, RWD, SW, true>(&cfg, attr, 2, nullptr);
-    cfg.numAttrs = 1;  // the occupancy query takes the cluster shape alone
-    cfg.attrs = attr + 1;
     if (cudaOccupancyMaxActiveClusters(&clusters, encode_flow_kernel<EW, RWD, SW, true, true, 8, true>, &cfg) !=
         cudaSuccess) {
       (void)cudaGetLastError();
@@ -2343,7 +2349,7 @@ template <int EPI, int RW, int SK, bool CB, bool XB, int NCH, bool PAIR = false>
 inline cudaError_t launch_flow_t(int grid, cudaStream_t s, const CUtensorMap &tmA0, const CUtensorMap &tmA,
                                  const CUtensorMap &tmB3, const GemmArgs &ga, const RowArgs &ra, const FlowArgs &fa) {
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   flow_launch_config<EPI, RW, SK, PAIR>(&cfg, attr, grid, s);
   return cudaLaunchKernelEx(&cfg, encode_flow_kernel<EPI, RW, SK, CB, XB, NCH, PAIR>, tmA0, tmA, tmB3, ga, ra, fa);
 }
