@@ -102,6 +102,17 @@ def test_bound_holds_on_packed_shaped_rows():
     print(f"packed-shaped: {entries} candidate scores, max |err|/E = {worst:.3g}")
 
 
+def test_bound_holds_with_cta_pairs():
+    """All-levels kernel run as CTA pairs (a batch of 65536+ rows at D = 1024): the M = 256 MMAs
+    of a pair must meet the same bound; rows from both CTAs of a pair are sampled."""
+    g = workloads.generate("packed", n_override=66000)
+    x, C = g["x"], np.ascontiguousarray(g["codebooks"][:3])
+    rows = workloads.sample_rows(len(x), 384, seed=35)
+    assert (((rows // 128) % 2) == 1).any() and (((rows // 128) % 2) == 0).any()
+    worst, entries = measure(x, C, "bf16", rows)
+    print(f"packed-shaped, CTA pairs: {entries} candidate scores, max |err|/E = {worst:.3g}")
+
+
 def test_bound_holds_on_offline_shaped_rows():
     """All-levels kernel, D = 256, K = 65536: level-1 candidates of mixture features."""
     g = workloads.generate("offline", n_override=8192)
