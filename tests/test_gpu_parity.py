@@ -95,11 +95,13 @@ def test_offline_sampled():
     assert (ids[:, 0] == g["planted"][:, 0]).mean() > 0.999   # mixture centre recovered
 
 
-def test_pairs_ragged_last_unit():
-    """A batch long enough for CTA pairs with an odd number of 128-row tiles (the last pair's
-    second tile holds no rows) and a ragged last codeword tile: sampled rows plus every row of the
-    last two row tiles against the oracle, properties on all rows."""
-    N, D, L, K = 65636, 1024, 3, 700
+@pytest.mark.parametrize("D,L,K", [(1024, 3, 700), (256, 2, 1500)])
+def test_pairs_ragged_last_unit(D, L, K):
+    """A batch long enough for CTA pairs with an odd number of 128-row tiles (at D = 1024 the last
+    pair's second tile holds no rows; D = 256 runs single CTAs) and a ragged last codeword tile:
+    sampled rows plus every row of the last two row tiles against the oracle, properties on all
+    rows."""
+    N = 65636
     rng = np.random.Generator(np.random.PCG64(4242))
     C = np.stack([rng.standard_normal((K, D), dtype=np.float32) * np.float32(0.5 ** l) for l in range(L)])
     planted = rng.integers(0, K, size=(N, L)).astype(np.int32)
