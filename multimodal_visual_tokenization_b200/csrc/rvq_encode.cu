@@ -2083,9 +2083,9 @@ struct Plan {
 
 // Smallest batch that the all-levels kernel runs as CTA pairs.  Pairs halve each SM's codeword
 // tile traffic and draw less power, which pays under the power cap of a long launch (2^20 rows
-// of D = 1024, L = 8, K = 16384: 222 vs 238 ms; 206181 rows, L = 8: 45 vs 46.5 ms); a launch
-// short enough to run at the boost clock (4096 rows) is faster with single CTAs.
-constexpr int64_t kPairMinRows = 65536;
+// of D = 1024, L = 8, K = 16384: 222 vs 238 ms; 206181 rows, L = 8: 45 vs 46.5 ms; 16352 rows:
+// 3.56-3.65 vs 3.70-3.72 ms); at 4096 rows (L = 4, K = 8192) the two run the same.
+constexpr int64_t kPairMinRows = 8192;
 
 inline bool flow_pairs_fit(int grid);
 

@@ -103,7 +103,7 @@ def test_bound_holds_on_packed_shaped_rows():
 
 
 def test_bound_holds_with_cta_pairs():
-    """All-levels kernel run as CTA pairs (a batch of 65536+ rows at D = 1024): the M = 256 MMAs
+    """All-levels kernel run as CTA pairs (66000 rows at D = 1024): the M = 256 MMAs
     of a pair must meet the same bound; rows from both CTAs of a pair are sampled."""
     g = workloads.generate("packed", n_override=66000)
     x, C = g["x"], np.ascontiguousarray(g["codebooks"][:3])

@@ -84,6 +84,19 @@ def test_packed_sampled():
     assert (ids[:, 0] == g["planted"][:, 0]).all()
 
 
+def test_packed_short_batch_pairs():
+    """A 16352-row packed batch runs as CTA pairs with several chunks per 256-row unit (so every
+    row merges several candidate lists written by a pair): sampled rows and every image boundary
+    against the oracle."""
+    g = workloads.generate("packed", n_override=16384)
+    x, C, off = g["x"], g["codebooks"], g["offsets"]
+    _, ids, res, rec, fb = run_encode(x, C, "bf16", "f32", offsets=off)
+    rows = workloads.sample_rows(len(x), 4096, seed=12, offsets=off)
+    rep = full_check(x, C, ids, res, rec, rows)
+    print("packed short", len(x), rep, "fallbacks", fb.tolist())
+    assert (ids[:, 0] == g["planted"][:, 0]).all()
+
+
 def test_offline_sampled():
     g = workloads.generate("offline")
     x, C = g["x"], g["codebooks"]
