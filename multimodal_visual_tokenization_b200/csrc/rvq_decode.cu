@@ -181,7 +181,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeBlocksPerSm) decode_
   int myid = (gl < LC && n < N) ? __ldg(ids + n * LC + gl) : 0;
   bool bad = false;
   while (true) {
-    const bool live = n < N;  // the warp's last rows may lie past N (never stored)
+    // with several rows per warp the last rows may lie past N (never stored); one row per warp
+    // never walks past N, and a constant keeps that loop free of the predicate
+    const bool live = RPW == 1 || n < N;
     Gather<CB_BF16, VEC> g[LC];
     bool use[LC];
 #pragma unroll
