@@ -15,15 +15,15 @@
 // row; the distance matrix never leaves the SM.
 //
 //  * encode_flow_kernel (D in (128, 256] or (512, 1024]): every level in ONE launch with every
-//    CTA resident (cooperative for single CTAs), one CTA per SM.  The level loop is a dataflow over 128-row tiles: GEMM chunks of (level l,
-//    row tile rt) start as soon as the certificate warps have settled level l-1 of rt (counter
-//    cert_done[l-1][rt]); the certificate warps take (l, rt) once all its chunks are written
-//    (chunk_done[l][rt]).  Per CTA: a TMA producer warp, an MMA-issuer warp, a norm-split warp,
-//    4 epilogue + 4 certificate warps (D in (512, 1024]) or 8 + 3 (D in (128, 256]).  For D in
-//    (512, 1024] and batches of at least kPairMinRows rows the CTAs run as pairs (2-CTA clusters,
-//    tcgen05 cta_group::2): each CTA loads its own 128 rows and half of every 256-codeword tile,
-//    the leader issues M = 256 MMAs, and each CTA's TMEM holds its own rows' accumulators, so an
-//    SM streams 32 KB instead of 48 KB per K step.  Rows the certificate cannot settle get an
+//    CTA resident (cooperative for single CTAs), one CTA per SM.  The level loop is a dataflow
+//    over 128-row tiles: GEMM chunks of (level l, row tile rt) start as soon as the certificate
+//    warps have settled level l-1 of rt (counter cert_done[l-1][rt]); the certificate warps take
+//    (l, rt) once all its chunks are written (chunk_done[l][rt]).  Per CTA: a TMA producer warp,
+//    an MMA-issuer warp, a norm-split warp, 4 epilogue + 4 certificate warps (D in (512, 1024]) or
+//    8 + 3 (D in (128, 256]).  For D in (512, 1024] and batches of at least kPairMinRows rows the
+//    CTAs run as pairs (2-CTA clusters, tcgen05 cta_group::2): each CTA loads its own 128 rows and
+//    half of every 256-codeword tile, the leader issues M = 256 MMAs, and each CTA's TMEM holds its
+//    own rows' accumulators, so an SM streams 32 KB instead of 48 KB per K step.  Rows the certificate cannot settle get an
 //    exact scan of all K codewords, cut into slices any certificate warp may run.  Every wait is
 //    bounded (status RVQ_ERR_TIMEOUT when nothing moved for two seconds).
 //  * other widths (and RVQ_PERSISTENT=0): per level, dist_topk_kernel (persistent GEMM + top-8 over
