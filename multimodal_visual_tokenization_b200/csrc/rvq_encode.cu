@@ -1234,14 +1234,15 @@ inline cudaError_t launch_rows_fast(const RowArgs &ra, int nch, unsigned row_blo
 }
 
 // ---------------------------------------------------------------- all levels in one launch
-// One cooperative launch runs every level as a dataflow over row tiles:
+// One launch with every CTA resident runs every level as a dataflow over row tiles:
 //
 //  * GEMM chunks.  Chunk (l, rt, j) scores row tile rt against codeword tiles [jS, (j+1)S) of
 //    level l and writes one partial top-8 list per row into slot j.  Chunks are numbered level by
-//    level, row tile by row tile, and CTA c takes chunks c, c+G, c+2G, ...  The TMA producer,
-//    MMA issuer, norm splitter and epilogue warps walk that sequence with the shared-memory ring,
-//    the TMEM buffers and the mbarrier phases carried from chunk to chunk.  Before loading chunk
-//    (l, rt, j) the producer waits until row tile rt is settled at level l-1.
+//    level, row tile by row tile, and CTA c takes chunks c, c+G, c+2G, ... (CTA pairs: pair c
+//    takes the chunks of 256-row units, each CTA scoring its own row tile of the unit).  The TMA
+//    producer, MMA issuer, norm splitter and epilogue warps walk that sequence with the
+//    shared-memory ring, the TMEM buffers and the mbarrier phases carried from chunk to chunk.
+//    Before loading chunk (l, rt, j) the producer waits until row tile rt is settled at level l-1.
 //  * Certificate tasks.  RW warps per CTA take tasks (l, rt, g) the same way (RPT rows each):
 //    once all NC chunks of (l, rt) are written they certify the rows, apply r -= C_l[id] and
 //    count the settled rows.  A row the certificate cannot settle goes to a queue whose exact
@@ -2071,7 +2072,7 @@ struct Plan {
   int64_t U;
   int G;       // CTAs
   int maxs;    // partial-list slots per row tile (the larger of the two paths' needs)
-  // all levels in one cooperative launch (encode_flow_kernel)
+  // all levels in one launch with every CTA resident (encode_flow_kernel)
   bool flow;
   int L;
   int NC, S;      // chunks per row tile, codeword tiles per chunk
@@ -2494,7 +2495,7 @@ extern "C" int rvq_encode(const void *features, int f_dtype, int64_t N, int D, c
   CUtensorMap tmX;
   if (x_is_operand && !make_map(&tmX, features, N, D, BM)) return RVQ_ERR_CUDA;
 
-  // D in (128, 256] or (512, 1024]: every level in one cooperative launch.
+  // D in (128, 256] or (512, 1024]: every level in one launch (CTA pairs for long batches at D > 512).
   const bool all_levels = fast && p.flow;
   if (all_levels) {
     if (!flow_attrs_ready()) return RVQ_ERR_CUDA;
