@@ -139,7 +139,8 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Tile loads of a CTA pair: the destination is this CTA's shared memory, the bytes are counted on
-// an mbarrier given as a shared::cluster address (the pair leader's).  No multicast.
+// an mbarrier given as a shared::cluster address (the pair leader's); each load fills only the
+// issuing CTA's own shared memory.
 __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, uint32_t bar_cluster_addr, void *dst,
                                                  int32_t x, int32_t y) {
   asm volatile(
