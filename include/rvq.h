@@ -165,6 +165,15 @@ RVQ_API int rvq_encode_noalloc(const void *features, int f_dtype, int64_t N, int
 RVQ_API int rvq_decode(const int32_t *ids, int64_t N, int L, const void *codebooks, int cb_dtype,
                int K, int D, float *recon, int32_t *status, void *stream);
 
+/*
+ * rvq_decode_slice_plan: how rvq_decode splits the work for this shape (host only, no device
+ * call).  A warp walks the rows of one column slice of `*slice_cols` columns with
+ * `*rows_per_warp` rows at a time (32 / rows_per_warp lanes per row); the slice narrows (2 or 4
+ * rows per warp) when its live codebook columns, L * K * slice_cols * element size, would exceed
+ * 64 MiB of L2.  Same argument checks as rvq_decode (RVQ_ERR_ARG for null outputs).
+ */
+RVQ_API int rvq_decode_slice_plan(int L, int K, int D, int cb_dtype, int *rows_per_warp, int *slice_cols);
+
 /* Human-readable name of an rvq_status value (static string). */
 RVQ_API const char *rvq_status_str(int status);
 

@@ -45,7 +45,7 @@ EXPORTS = ("rvq_build_norms", "rvq_encode_workspace_size", "rvq_encode", "rvq_de
            "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
            "rvq_encode_noalloc", "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply",
            "rvq_ipc_export", "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
-           "rvq_embed_backward_sorted", "rvq_encode_candidate_layout")
+           "rvq_embed_backward_sorted", "rvq_encode_candidate_layout", "rvq_decode_slice_plan")
 RVQ_MAX_SHARDS = 16
 RVQ_IPC_HANDLE_BYTES = 64
 RVQ_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -87,6 +87,7 @@ def load():
         lib.rvq_profile_read.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double)]
         lib.rvq_encode_levels_per_launch.argtypes = [i64, i32, i32, i32, ctypes.POINTER(i32)]
         lib.rvq_encode_candidate_layout.argtypes = [i64, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(i32)]
+        lib.rvq_decode_slice_plan.argtypes = [i32, i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
         lib.rvq_selftest_wait_timeout.argtypes = [vp, vp, i64, vp]
         lib.rvq_embed_backward.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp, vp]
         lib.rvq_codebook_update.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -108,7 +109,7 @@ def load():
                    "rvq_codebook_update", "rvq_balance_sequences", "rvq_gather_sequences",
                    "rvq_shard_workspace_size", "rvq_shard_select", "rvq_shard_apply", "rvq_ipc_export",
                    "rvq_ipc_import", "rvq_ipc_close", "rvq_embed_backward_workspace_size",
-                   "rvq_embed_backward_sorted", "rvq_encode_candidate_layout"):
+                   "rvq_embed_backward_sorted", "rvq_encode_candidate_layout", "rvq_decode_slice_plan"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -214,6 +215,14 @@ def rvq_encode_candidate_layout(N, D, L, K):
     slots = ctypes.c_int32(0)
     code = load().rvq_encode_candidate_layout(int(N), int(D), int(L), int(K), ctypes.byref(off), ctypes.byref(slots))
     return code, off.value, slots.value
+
+
+def rvq_decode_slice_plan(L, K, D, cb_dtype):
+    """-> (status, rows per warp, columns per slice) that rvq_decode uses for this shape."""
+    rpw = ctypes.c_int32(0)
+    cols = ctypes.c_int32(0)
+    code = load().rvq_decode_slice_plan(int(L), int(K), int(D), int(cb_dtype), ctypes.byref(rpw), ctypes.byref(cols))
+    return code, rpw.value, cols.value
 
 
 def rvq_embed_backward(ids, N, L, K, H, grad_out, grad_tables, status=None, stream=None):

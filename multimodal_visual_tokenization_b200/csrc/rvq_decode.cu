@@ -304,6 +304,22 @@ int launch_decode(const int32_t *ids, int64_t N, int L, const void *cb, int cb_d
 
 }  // namespace rvq
 
+extern "C" int rvq_decode_slice_plan(int L, int K, int D, int cb_dtype, int *rows_per_warp, int *slice_cols) {
+  using namespace rvq;
+  if (!rows_per_warp || !slice_cols) return RVQ_ERR_ARG;
+  if (L < 1 || K < 1 || D < 1) return RVQ_ERR_ARG;
+  if (cb_dtype != RVQ_F32 && cb_dtype != RVQ_BF16) return RVQ_ERR_ARG;
+  if (L > 64 || D < 4 || D % 4 != 0) return RVQ_ERR_UNSUPPORTED;
+  const int vec = (cb_dtype == RVQ_BF16 && D % 8 == 0) ? 8 : 4;
+  const int elem = cb_dtype == RVQ_BF16 ? 2 : 4;
+  // the same choice launch_decode makes: rows per warp for the fixed-level kernel, one row per warp
+  // in the generic kernel (more than 16 levels)
+  const int rpw = L <= 16 ? decode_rows_per_warp(L, K, vec, elem) : 1;
+  *rows_per_warp = rpw;
+  *slice_cols = 32 / rpw * vec;
+  return RVQ_OK;
+}
+
 extern "C" int rvq_decode(const int32_t *ids, int64_t N, int L, const void *codebooks, int cb_dtype, int K, int D,
                           float *recon, int32_t *status, void *stream) {
   RVQ_ENTRY("rvq_decode");

@@ -146,6 +146,44 @@ def test_host_argument_checks(lib):
     assert ebs(16, 5, 2, 8, 16, 16, 16, 256, 100, None, None) == -3                         # too small
 
 
+@pytest.mark.parametrize("L,K,D,dt,want_rpw,want_cols", [
+    (8, 16384, 1024, "bf16", 1, 256),   # detok: 8 x 16384 x 256 bf16 columns = 64 MiB live
+    (8, 16384, 1024, "f32", 1, 128),    # packed: 64 MiB
+    (4, 8192, 1024, "f32", 1, 128),     # image: 16 MiB
+    (4, 65536, 256, "f32", 2, 64),      # offline: 128 MiB at 128 columns, 64 MiB at 64
+    (8, 65536, 128, "f32", 4, 32),      # 256 MiB -> 128 -> 64 MiB
+    (8, 65536, 256, "bf16", 4, 64),     # bf16, 16-byte gathers
+    (12, 32768, 132, "bf16", 2, 64),    # D % 8 != 0: 8-byte gathers; 12 levels fit 16 lanes, not 8
+    (16, 65536, 256, "f32", 2, 64),     # 16 levels: at most two rows per warp
+    (20, 65536, 256, "f32", 1, 128),    # more than 16 levels: the generic kernel, one row per warp
+    (1, 7, 256, "bf16", 1, 256),
+])
+def test_decode_slice_plan(lib, L, K, D, dt, want_rpw, want_cols):
+    """The rows-per-warp choice of rvq_decode: the widest slice whose live codebook columns
+    (L * K * columns * element size) stay within 64 MiB, as narrow as a row's ids allow."""
+    code, rpw, cols = mvt.rvq_decode_slice_plan(L, K, D, mvt.RVQ_BF16 if dt == "bf16" else mvt.RVQ_F32)
+    assert code == 0 and (rpw, cols) == (want_rpw, want_cols)
+    el = 2 if dt == "bf16" else 4
+    if L <= 16:
+        lanes = 32 // rpw
+        assert L <= lanes
+        live = L * K * cols * el
+        narrower_allowed = rpw < 4 and L <= lanes // 2
+        assert live <= 64 << 20 or not narrower_allowed
+        if rpw > 1:  # one step wider would have exceeded the budget
+            assert L * K * (cols * 2) * el > 64 << 20
+
+
+def test_decode_slice_plan_argument_checks(lib):
+    i32 = ctypes.c_int32
+    a, b = i32(0), i32(0)
+    assert lib.rvq_decode_slice_plan(8, 16384, 1024, 1, None, ctypes.byref(b)) == -1
+    assert lib.rvq_decode_slice_plan(0, 16384, 1024, 1, ctypes.byref(a), ctypes.byref(b)) == -1
+    assert lib.rvq_decode_slice_plan(8, 16384, 1024, 7, ctypes.byref(a), ctypes.byref(b)) == -1
+    assert lib.rvq_decode_slice_plan(8, 16384, 1022, 1, ctypes.byref(a), ctypes.byref(b)) == -2
+    assert lib.rvq_decode_slice_plan(65, 16384, 1024, 1, ctypes.byref(a), ctypes.byref(b)) == -2
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     """No CPU fallback: without librvq.so the binding raises instead of running anything else."""
     monkeypatch.setattr(mvt, "_lib", None)
