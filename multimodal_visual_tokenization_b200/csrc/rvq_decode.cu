@@ -8,6 +8,9 @@
 // slice-major (blockIdx.y = slice), so while one slice is being produced only L*K*slice codebook
 // elements are live and stay resident in L2; recon is written with streaming stores.  Gathers of
 // all levels of a row are in flight at once per warp, and the next row's ids are fetched meanwhile.
+// When a slice's live codebook columns would exceed 64 MiB, two or four rows share a warp and the
+// slice narrows to a half or a quarter (fp32 codebooks of 4 x 65536 codewords at D = 256: 0.55 vs
+// 0.83 ms); rvq_decode_slice_plan reports the choice.
 //
 // Measured bound (2^20 tokens, 8 levels, [8,16384,1024] bf16): the L2 -> SM delivery of the gathered
 // rows, ~10 TB/s for 512-byte row pieces.  A gather-only copy of this kernel takes about as long as
