@@ -24,6 +24,8 @@ Other entry points:
 * ``rvq_balance_sequences`` / ``rvq_gather_sequences``: packing id sequences for data-parallel
   ranks.
 * ``sharded.ShardedTokenizer``: the codebook axis split over the ranks of a process group.
+* Queries and measurement hooks: ``rvq_encode_levels_per_launch``, ``rvq_encode_candidate_layout``,
+  ``rvq_decode_slice_plan``, ``rvq_launch_count``, ``rvq_profile_enable`` / ``rvq_profile_read``.
 """
 from __future__ import annotations
 
